@@ -1,0 +1,394 @@
+"""Benchmark of the attention hot path on B200.
+
+Default workload (one GPU): the 8B-shaped packed prefill, B=4, S=8192, Hq=32,
+Hkv=8, D=128, bf16, causal + cross-document mask with documents U[512, 4096].
+One step is one llama_attn_prefill call over that batch (document layout,
+K rotation, tensor-core attention). The metric counts only unmasked (i, j)
+pairs: FLOPs = 4 * D * Hq * pairs. The decode form of the hot path (70B-shaped,
+64 sequences, Hq=64, Hkv=8, cache lengths U[1024, 32768]) is measured in the
+same run after the timed prefill steps and reported under "decode" (GB/s of
+cached K/V rows read).
+
+`--impl reference` times the float64 CPU oracle on the host cores instead, on
+a bounded sample of query rows of the same workload, in the same unit.
+
+Multi-GPU (torchrun): one process per GPU, each with its own independent
+batch (weak scaling, no data-path collective); rank 0 prints the line, value =
+FLOPs of all ranks / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gqa_attention_rope_b200 import workloads as W  # noqa: E402
+
+METRIC = "prefill attention TFLOP/s (causal) & decode KV-cache GB/s, % of B200 roofline"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained", 0)), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling while the timed region runs."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{self.index}.csv")
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- CPU oracle baseline
+
+def oracle_rows_sample(w, inp, target_s: float, seed: int = 99):
+    """Time the float64 oracle on growing samples of query rows until about
+    target_s seconds of work; returns (flops_done, seconds, n_rows, threads)."""
+    from oracle import oracle as O
+    lay = O.doc_layout(inp["doc_offsets"], w.B, w.S)
+    ds = lay[0].astype(np.int64)
+    g = np.random.default_rng(seed)
+    n = 8
+    while True:
+        rows = np.sort(g.choice(w.B * w.S, size=n, replace=False))
+        t0 = time.perf_counter()
+        O.prefill(inp["q"], inp["k"], inp["v"], inp["doc_offsets"], w.rope_theta, rows=rows, layout=lay)
+        dt = time.perf_counter() - t0
+        visible = ((rows % w.S) - ds[rows] + 1).sum()  # keys each sampled row attends to
+        flops = 4.0 * w.D * w.Hq * float(visible)
+        if dt >= target_s or n >= w.B * w.S // 2:
+            return flops, dt, n, O.num_threads()
+        n = int(min(w.B * w.S // 2, max(2 * n, n * target_s / max(dt, 1e-3))))
+
+
+def run_reference(args, w):
+    """The oracle as the reference arm: each step is a bounded sample of rows."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = W.make_prefill_inputs(w)
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_rows_sample(w, inp, per_step / 4)
+    flops = secs = 0.0
+    rows = threads = 0
+    for _ in range(args.steps):
+        f, s, n, threads = oracle_rows_sample(w, inp, per_step)
+        flops += f
+        secs += s
+        rows += n
+    value = flops / secs / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, world),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} random query rows x {w.Hq} heads of {w.name} over {args.steps} steps "
+                                   "(float64 C oracle, OpenMP, full masked rows)"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, world):
+    return {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+            "doc_lengths": None if w.doc_range is None else f"U[{w.doc_range[0]},{w.doc_range[1]}]",
+            "rope_theta": w.rope_theta, "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)",
+            "parallelism": f"{world} independent replicas (weak scaling)" if world > 1 else "1 GPU"}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_ours(args, w):
+    import gqa_attention_rope_b200 as la
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    la.lib()
+    hbm_peak, tc_peak, tc_sust, peak_kind = load_peaks()
+
+    # inputs: per-rank seed so ranks hold independent batches
+    wr = W.PrefillWorkload(w.name, w.seed + 1000 * rank, w.B, w.S, w.Hq, w.Hkv, w.D, w.dtype, w.doc_range,
+                           w.rope_theta)
+    inp = W.make_prefill_inputs(wr)
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    offs = inp["doc_offsets"].to(dev) if inp["doc_offsets"] is not None else None
+    out = torch.empty_like(q)
+    pairs = W.unmasked_pairs(inp["doc_offsets"], wr.B, wr.S)
+    flops = 4.0 * w.D * w.Hq * pairs
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        la.llama_attn_prefill(q, k, v, out=out, doc_offsets=offs, rope_theta=w.rope_theta)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if la.llama_attn_get_device_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    la.llama_attn_profile_begin()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    main_ms, main_n, launches = la.llama_attn_profile_end()
+    barrier(world)
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    all_flops = sum_over_ranks(flops * args.steps, world)
+    value = all_flops / (total_ms / 1e3) / 1e12
+    kernel_ms = main_ms / max(main_n, 1)
+    achieved = flops / (kernel_ms / 1e3) / 1e12
+
+    # end to end through the public API: pinned host inputs -> device -> call -> host result
+    hq, hk, hv = (inp[n].pin_memory() for n in ("q", "k", "v"))
+    hoffs = inp["doc_offsets"].pin_memory() if inp["doc_offsets"] is not None else None
+    hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+    dq, dk, dv, dout = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(q)
+    doffs = torch.empty_like(offs) if offs is not None else None
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        if doffs is not None:
+            doffs.copy_(hoffs, non_blocking=True)
+        la.llama_attn_prefill(dq, dk, dv, out=dout, doc_offsets=doffs, rope_theta=w.rope_theta)
+        hout.copy_(dout, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    for i in range(args.steps):
+        e_ev[i][0].record(stream)
+        e2e_step()
+        e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev), world)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv)) + (hoffs.numel() * 4 if hoffs is not None else 0)
+    d2h = hout.numel() * hout.element_size()
+    e2e = {"value": all_flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h}
+    del hq, hk, hv, hout, dq, dk, dv, dout
+
+    decode = None if args.no_decode else run_decode(args, la, dev, world, rank, hbm_peak, peak_kind)
+    if la.llama_attn_get_device_error() != 0:
+        raise RuntimeError("device error word set during the benchmark")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, s, n, threads = oracle_rows_sample(wr, inp, args.cpu_seconds)
+        cpu = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} random query rows x {w.Hq} heads of {w.name} (float64 C oracle, "
+                         f"full masked rows, {s:.1f} s)"}
+
+    traffic = load_traffic("prefill_bf16_kernel", w.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(config_of(w, world), flops_per_step_per_gpu=flops, unmasked_pairs_per_head=pairs),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                     "frac": achieved / tc_peak, "peak_kind": f"{peak_kind} bf16 dense (burst)",
+                     "kernel": "prefill_bf16_kernel", "kernel_ms": kernel_ms, "traffic": traffic},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": clk,
+        "gpu_launches": launches + (decode["gpu_launches"] if decode else 0),
+        "decode": decode,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_decode(args, la, dev, world, rank, hbm_peak, peak_kind):
+    w = W.DECODE_70B
+    wr = W.DecodeWorkload(w.name, w.seed + 1000 * rank, w.B, w.Hq, w.Hkv, w.D, w.Lmax, w.len_range)
+    inp = W.make_decode_inputs(wr, poison=True)
+    q, kc, vc, lens = (inp[n].to(dev) for n in ("q", "kcache", "vcache", "cache_lens"))
+    del inp["kcache"], inp["vcache"]
+    out = torch.empty_like(q)
+    ws = torch.empty(la.llama_attn_decode_workspace_size(w.B, w.Hq, w.Lmax, w.D), dtype=torch.uint8, device=dev)
+    tokens = W.cache_tokens(inp["cache_lens"])
+    kv_bytes = tokens * w.Hkv * w.D * 2 * 2
+    io_bytes = q.numel() * 2 * 2 + lens.numel() * 4
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        la.llama_attn_decode(q, kc, vc, lens, out=out, workspace=ws, rope_theta=w.rope_theta)
+
+    for _ in range(5):
+        step()
+    torch.cuda.synchronize()
+    steps = max(args.steps, 10)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier(world)
+    la.llama_attn_profile_begin()
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    main_ms, main_n, launches = la.llama_attn_profile_end()
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world)
+    all_bytes = sum_over_ranks(float(kv_bytes + io_bytes) * steps, world)
+    kernel_ms = main_ms / max(main_n, 1)
+    achieved = kv_bytes / (kernel_ms / 1e3) / 1e9
+    return {
+        "workload": w.name, "value": all_bytes / (total_ms / 1e3) / 1e9, "unit": "GB/s", "steps": steps,
+        "ms_per_step": total_ms / steps, "bytes_per_step_per_gpu": kv_bytes + io_bytes, "cache_tokens": tokens,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "peak_kind": f"{peak_kind} HBM copy",
+                     "kernel": "decode_split_kernel", "kernel_ms": kernel_ms,
+                     "traffic": load_traffic("decode_split_kernel", w.name)},
+        "gpu_launches": launches,
+    }
+
+
+def load_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if one matches."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        return t[kernel][workload]
+    except Exception:
+        return None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=W.PACKED_8B.name, choices=[n for n, x in W.WORKLOADS.items()
+                                                                      if isinstance(x, W.PrefillWorkload)])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    w = W.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        if w.dtype != "bf16":
+            raise SystemExit("the bench times the bf16 tensor-core path")
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,204 @@
+"""Python binding of the B200 attention library (libllama_attn.so).
+
+The functions carry the names of the C ABI in include/llama_attn.h and only
+marshal arguments: shapes are read off the tensors, device pointers and the
+current CUDA stream are passed through ctypes, and a negative status becomes
+a RuntimeError. Every step of the computation runs in the library's CUDA
+kernels; there is no CPU or PyTorch fallback, and calling an op without the
+built library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libllama_attn.so")
+
+EXPORTED = (
+    "llama_attn_prefill",
+    "llama_attn_prefill_f32",
+    "llama_attn_decode_workspace_size",
+    "llama_attn_decode",
+    "llama_attn_status_string",
+    "llama_attn_get_device_error",
+    "llama_attn_version",
+    "llama_attn_profile_begin",
+    "llama_attn_profile_end",
+)
+
+DEVERR_TIMEOUT = 0x1
+DEVERR_DOC_OFFSETS = 0x2
+DEVERR_CACHE_LEN = 0x4
+
+_lock = threading.Lock()
+_lib = None
+
+
+class LlamaAttnError(RuntimeError):
+    def __init__(self, fn: str, status: int, text: str):
+        super().__init__(f"{fn} failed: status {status} ({text})")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the shared library and declare the C signatures. Raises if missing."""
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"libllama_attn.so not found at {path}; build it with "
+            "`python -m gqa_attention_rope_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(path)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.llama_attn_prefill.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P]
+    lib.llama_attn_prefill.restype = I
+    lib.llama_attn_prefill_f32.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P]
+    lib.llama_attn_prefill_f32.restype = I
+    lib.llama_attn_decode_workspace_size.argtypes = [I, I, I, I]
+    lib.llama_attn_decode_workspace_size.restype = Z
+    lib.llama_attn_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P, Z, P]
+    lib.llama_attn_decode.restype = I
+    lib.llama_attn_status_string.argtypes = [I]
+    lib.llama_attn_status_string.restype = ctypes.c_char_p
+    lib.llama_attn_get_device_error.argtypes = [P]
+    lib.llama_attn_get_device_error.restype = I
+    lib.llama_attn_version.argtypes = []
+    lib.llama_attn_version.restype = I
+    lib.llama_attn_profile_begin.argtypes = []
+    lib.llama_attn_profile_begin.restype = I
+    lib.llama_attn_profile_end.argtypes = [P, P, P]
+    lib.llama_attn_profile_end.restype = I
+    return lib
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = load_library()
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise LlamaAttnError(fn, status, lib().llama_attn_status_string(status).decode())
+
+
+def _require(cond: bool, msg: str):
+    if not cond:
+        raise ValueError(msg)
+
+
+def llama_attn_status_string(status: int) -> str:
+    return lib().llama_attn_status_string(int(status)).decode()
+
+
+def llama_attn_version() -> int:
+    return int(lib().llama_attn_version())
+
+
+def llama_attn_get_device_error(stream=None) -> int:
+    st = lib().llama_attn_get_device_error(_stream(stream))
+    if st < 0:
+        _check("llama_attn_get_device_error", st)
+    return st
+
+
+def llama_attn_profile_begin() -> None:
+    _check("llama_attn_profile_begin", lib().llama_attn_profile_begin())
+
+
+def llama_attn_profile_end():
+    """Returns (main_kernel_ms_total, main_kernels_timed, kernels_launched)."""
+    ms = ctypes.c_double(0.0)
+    n_main = ctypes.c_int(0)
+    n_all = ctypes.c_int(0)
+    _check("llama_attn_profile_end", lib().llama_attn_profile_end(ctypes.byref(ms), ctypes.byref(n_main),
+                                                                 ctypes.byref(n_all)))
+    return ms.value, n_main.value, n_all.value
+
+
+def llama_attn_prefill(q, k, v, out=None, doc_offsets=None, rope_theta: float = 500000.0, stream=None):
+    """bf16 prefill. q [B,S,Hq,D], k/v [B,S,Hkv,D] contiguous CUDA bf16; returns out [B,S,Hq,D]."""
+    import torch
+    _require(q.dim() == 4 and k.dim() == 4 and v.dim() == 4, "q, k, v must be [B, S, H, D]")
+    for t in (q, k, v):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "bf16 contiguous CUDA tensors expected")
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _require(k.shape == (B, S, Hkv, D) and v.shape == k.shape, "k and v must be [B, S, Hkv, D]")
+    if out is None:
+        out = torch.empty_like(q)
+    _require(out.shape == q.shape and out.dtype == torch.bfloat16 and out.is_contiguous(), "bad out")
+    if doc_offsets is not None:
+        _require(doc_offsets.is_cuda and doc_offsets.dtype == torch.int32, "doc_offsets: int32 CUDA tensor")
+    st = lib().llama_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(doc_offsets), B, S, Hq, Hkv, D,
+                                  float(rope_theta), _stream(stream))
+    _check("llama_attn_prefill", st)
+    return out
+
+
+def llama_attn_prefill_f32(q, k, v, out=None, doc_offsets=None, rope_theta: float = 500000.0, stream=None):
+    """fp32 prefill on CUDA cores; same layout as llama_attn_prefill with float32 tensors."""
+    import torch
+    _require(q.dim() == 4 and k.dim() == 4 and v.dim() == 4, "q, k, v must be [B, S, H, D]")
+    for t in (q, k, v):
+        _require(t.is_cuda and t.dtype == torch.float32 and t.is_contiguous(), "f32 contiguous CUDA tensors expected")
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _require(k.shape == (B, S, Hkv, D) and v.shape == k.shape, "k and v must be [B, S, Hkv, D]")
+    if out is None:
+        out = torch.empty_like(q)
+    if doc_offsets is not None:
+        _require(doc_offsets.is_cuda and doc_offsets.dtype == torch.int32, "doc_offsets: int32 CUDA tensor")
+    st = lib().llama_attn_prefill_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(doc_offsets), B, S, Hq, Hkv, D,
+                                      float(rope_theta), _stream(stream))
+    _check("llama_attn_prefill_f32", st)
+    return out
+
+
+def llama_attn_decode_workspace_size(B: int, Hq: int, Lmax: int, D: int = 128) -> int:
+    return int(lib().llama_attn_decode_workspace_size(B, Hq, Lmax, D))
+
+
+def llama_attn_decode(q, kcache, vcache, cache_lens, out=None, workspace=None, rope_theta: float = 500000.0,
+                      stream=None):
+    """bf16 decode. q [B,Hq,D]; kcache/vcache [B,Hkv,Lmax,D] (keys pre-rotated); cache_lens int32 [B]."""
+    import torch
+    _require(q.dim() == 3 and kcache.dim() == 4 and vcache.shape == kcache.shape, "bad shapes")
+    for t in (q, kcache, vcache):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "bf16 contiguous CUDA tensors expected")
+    _require(cache_lens.is_cuda and cache_lens.dtype == torch.int32, "cache_lens: int32 CUDA tensor")
+    B, Hq, D = q.shape
+    Hkv, Lmax = kcache.shape[1], kcache.shape[2]
+    _require(kcache.shape == (B, Hkv, Lmax, D) and cache_lens.numel() == B, "bad shapes")
+    if out is None:
+        out = torch.empty_like(q)
+    need = llama_attn_decode_workspace_size(B, Hq, Lmax, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib().llama_attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(cache_lens), _ptr(out), B, Hq, Hkv, D,
+                                 Lmax, float(rope_theta), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                 _stream(stream))
+    _check("llama_attn_decode", st)
+    return out
+
+
+def shard_units(n_units: int, world_size: int, rank: int):
+    """Contiguous, balanced split of independent work units (e.g. (batch row,
+    KV group) pairs of a prefill, or sequences of a decode) over ranks."""
+    if world_size <= 0 or not (0 <= rank < world_size):
+        raise ValueError("bad world_size / rank")
+    base, extra = divmod(n_units, world_size)
+    start = rank * base + min(rank, extra)
+    return range(start, start + base + (1 if rank < extra else 0))

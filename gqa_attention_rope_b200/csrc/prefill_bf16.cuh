@@ -1,0 +1,392 @@
+// prefill_bf16.cuh -- grouped-query causal attention with RoPE and the
+// cross-document mask on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// One CTA computes a 128-row query tile for NH (1 or 2) query heads of the same
+// KV group, so every K/V tile brought in by TMA serves both heads (GQA reuse).
+//
+//   warp 0      TMA producer: Q tiles once, then K/V tiles through a 3-stage ring
+//               in the order the MMA warp consumes them (K0, K1, V0, K2, V1, ...).
+//   warp 1      TMEM owner and single-thread MMA issuer:
+//                 S_h = Q_h K_j^T   (M=128, N=128, K=128; accumulators in TMEM)
+//                 O_h += P_h V_j    (P from shared memory, V MN-major)
+//   warps 4-7   softmax for head slot 0, warps 8-11 for slot 1: thread = query
+//               row = TMEM lane. Rotates its Q row in shared memory (RoPE at the
+//               row's document position), then per KV tile: S from TMEM ->
+//               registers, mask, row max, P = 2^(S*log2e/sqrt(D) - m) in bf16 to
+//               shared memory, running sum; O in TMEM is rescaled only when the
+//               running max grows by more than 2^8 (exact: the final 1/l uses the
+//               same reference max); epilogue O/l -> bf16 -> TMA store.
+//
+// TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
+// Shared memory (1024-aligned): Q_0, Q_1 (32 KB each), K/V ring 3 x 32 KB,
+// P_0, P_1 (32 KB each), barriers. Every 32 KB tile is two 64-column halves of
+// 128 rows x 128 B in the 128B-swizzled layout TMA writes.
+//
+// KV tiles run from the tile holding the document start of the first query
+// row to the diagonal tile; tiles entirely before that start are never loaded
+// or multiplied. Only tiles on the diagonal or before the last row's document
+// start apply the element mask.
+//
+// Keys arrive already rotated (a separate streaming pass writes RoPE(K) once
+// per key, which is cheaper than re-rotating every K tile for every query tile
+// that reads it).
+#pragma once
+
+#include "ptx.cuh"
+#include "rope.cuh"
+
+namespace la {
+namespace pfx {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int NSTAGE = 3;
+constexpr uint32_t TILE = 32768;
+constexpr uint32_t HALF = 16384;
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_KV = OFF_Q + 2 * TILE;
+constexpr uint32_t OFF_P = OFF_KV + NSTAGE * TILE;
+constexpr uint32_t OFF_BAR = OFF_P + 2 * TILE;
+constexpr uint32_t SMEM_USED = OFF_BAR + 256;
+constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;
+constexpr int NTHREADS = 384;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr float kRescaleLog2 = 8.0f;
+
+enum : int {
+  B_KV_FULL = 0,
+  B_KV_EMPTY = B_KV_FULL + NSTAGE,
+  B_Q_FULL = B_KV_EMPTY + NSTAGE,
+  B_Q_READY,
+  B_S_READY = B_Q_READY + 2,
+  B_S_FREE = B_S_READY + 2,
+  B_P_READY = B_S_FREE + 2,
+  B_PV_DONE = B_P_READY + 2,
+  B_O_STAGED = B_PV_DONE + 2,
+  B_DRAIN = B_O_STAGED + 2,
+  N_BARS
+};
+static_assert(N_BARS * 8 + 8 <= 256, "barrier area");
+
+struct Params {
+  int B, S, Hq, Hkv, G, NH, n_qt, n_hp;
+  const int32_t* doc_start;  // [B*S] row-local document start, or null (one document per row)
+  const float4* rope_tab;    // (cos, sin) pairs, 64 per position, as float4 = 2 pairs
+  float scale_log2;          // log2(e) / sqrt(D)
+  unsigned int epoch;        // launch id for bounded-wait abort propagation
+};
+
+__device__ __forceinline__ uint64_t kdesc(uint32_t saddr) { return umma_desc_sw128(saddr, 16, 1024); }
+__device__ __forceinline__ uint64_t vdesc(uint32_t saddr) { return umma_desc_sw128(saddr, HALF, 1024); }
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    prefill_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                        const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t bar0 = sbase + OFF_BAR;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * N_BARS);
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const WaitCtx wc{p.epoch};
+
+  // ---- work item: heaviest (highest) query tiles first
+  const int per_rank = p.B * p.n_hp;
+  const int qt = p.n_qt - 1 - static_cast<int>(blockIdx.x) / per_rank;
+  const int rem = static_cast<int>(blockIdx.x) % per_rank;
+  const int b = rem / p.n_hp, hp = rem % p.n_hp;
+  const int h0 = hp * p.NH;
+  const int g = h0 / p.G;
+  const int q0 = qt * BM;
+  const int q_last = min(q0 + BM - 1, p.S - 1);
+  const int64_t rowbase = static_cast<int64_t>(b) * p.S;
+  const int ds_first = p.doc_start ? p.doc_start[rowbase + q0] : 0;
+  const int ds_last = p.doc_start ? p.doc_start[rowbase + q_last] : 0;
+  const int kv_t0 = ds_first / BN;
+  const int n_kv = qt - kv_t0 + 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(bar(B_KV_FULL + s), 1);
+      mbar_init(bar(B_KV_EMPTY + s), 1);
+    }
+    mbar_init(bar(B_Q_FULL), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(B_Q_READY + s), 128);
+      mbar_init(bar(B_S_READY + s), 1);
+      mbar_init(bar(B_S_FREE + s), 128);
+      mbar_init(bar(B_P_READY + s), 128);
+      mbar_init(bar(B_PV_DONE + s), 1);
+      mbar_init(bar(B_O_STAGED + s), 128);
+    }
+    mbar_init(bar(B_DRAIN), 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_o);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(B_Q_FULL), static_cast<uint32_t>(p.NH) * TILE);
+      for (int s = 0; s < p.NH; ++s)
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_4d(sbase + OFF_Q + s * TILE + hf * HALF, &tm_q, bar(B_Q_FULL), hf * 64, h0 + s, q0, b);
+      uint32_t idx = 0;
+      auto load = [&](const CUtensorMap* tm, int kv_row) -> bool {
+        const uint32_t st = idx % NSTAGE, use = idx / NSTAGE;
+        if (use > 0 && !mbar_wait(bar(B_KV_EMPTY + st), (use - 1) & 1, wc)) return false;
+        mbar_arrive_expect_tx(bar(B_KV_FULL + st), TILE);
+        tma_load_4d(sbase + OFF_KV + st * TILE, tm, bar(B_KV_FULL + st), 0, g, kv_row, b);
+        tma_load_4d(sbase + OFF_KV + st * TILE + HALF, tm, bar(B_KV_FULL + st), 64, g, kv_row, b);
+        ++idx;
+        return true;
+      };
+      bool ok = load(&tm_k, kv_t0 * BN);
+      for (int j = 1; ok && j < n_kv; ++j)
+        ok = load(&tm_k, (kv_t0 + j) * BN) && load(&tm_v, (kv_t0 + j - 1) * BN);
+      if (ok) load(&tm_v, (kv_t0 + n_kv - 1) * BN);
+      // Every issued load has landed before this CTA may exit (returns at once
+      // in the normal flow, where the MMA warp consumed them all).
+      mbar_wait(bar(B_Q_FULL), 0, wc);
+      for (uint32_t st = 0; st < NSTAGE; ++st)
+        if (idx > st) mbar_wait(bar(B_KV_FULL + st), ((idx - 1 - st) / NSTAGE) & 1, wc);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = umma_idesc_bf16_f32(128, 128, 0);
+      constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 128, 1);
+      uint32_t idx = 0;
+      bool ok = true;
+      for (int s = 0; s < p.NH; ++s) ok = ok && mbar_wait(bar(B_Q_READY + s), 0, wc);
+      auto next = [&](uint32_t& st) -> bool {
+        st = idx % NSTAGE;
+        const uint32_t use = idx / NSTAGE;
+        ++idx;
+        const bool r = mbar_wait(bar(B_KV_FULL + st), use & 1, wc);
+        tc_fence_after();
+        return r;
+      };
+      auto issue_s = [&](int j, uint32_t st) -> bool {
+        for (int s = 0; s < p.NH; ++s) {
+          if (j > 0 && !mbar_wait(bar(B_S_FREE + s), (j - 1) & 1, wc)) return false;
+          tc_fence_after();
+          const uint32_t qa = sbase + OFF_Q + s * TILE, kb = sbase + OFF_KV + st * TILE;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
+            tc_mma_ss(tmem + s * 128, kdesc(qa + off), kdesc(kb + off), idesc_qk, kk > 0);
+          }
+          tc_commit(bar(B_S_READY + s));
+        }
+        tc_commit(bar(B_KV_EMPTY + st));
+        return true;
+      };
+      auto issue_pv = [&](int j, uint32_t st) -> bool {
+        for (int s = 0; s < p.NH; ++s) {
+          if (!mbar_wait(bar(B_P_READY + s), j & 1, wc)) return false;
+          tc_fence_after();
+          const uint32_t pa = sbase + OFF_P + s * TILE, vb = sbase + OFF_KV + st * TILE;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t aoff = (kk >> 2) * HALF + (kk & 3) * 32;
+            tc_mma_ss(tmem + 256 + s * 128, kdesc(pa + aoff), vdesc(vb + kk * 2048), idesc_pv,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(bar(B_PV_DONE + s));
+        }
+        tc_commit(bar(B_KV_EMPTY + st));
+        return true;
+      };
+      if (ok) {
+        uint32_t st;
+        ok = next(st) && issue_s(0, st);
+        for (int j = 1; ok && j < n_kv; ++j) {
+          ok = next(st) && issue_s(j, st);
+          ok = ok && next(st) && issue_pv(j - 1, st);
+        }
+        if (ok) ok = next(st) && issue_pv(n_kv - 1, st);
+      }
+      // all issued MMAs complete before TMEM may be freed
+      tc_commit(bar(B_DRAIN));
+      mbar_wait(bar(B_DRAIN), 0, wc);
+    }
+  } else if (warp >= 4 && (warp - 4) / 4 < p.NH) {
+    // ------------------------------------------------------------ softmax
+    const int s = (warp - 4) >> 2;
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + s * 128;
+    const uint32_t tO = tmem + lane_off + 256 + s * 128;
+    const int qi = q0 + r;
+    const bool row_valid = qi < p.S;
+    const int qi_c = min(qi, p.S - 1);
+    const int ds_i = p.doc_start ? p.doc_start[rowbase + qi_c] : 0;
+    uint8_t* qtile = smem + OFF_Q + s * TILE;
+    uint8_t* ptile = smem + OFF_P + s * TILE;
+
+    bool ok = mbar_wait(bar(B_Q_FULL), 0, wc);
+    if (ok && row_valid) {
+      const float4* tab = p.rope_tab + static_cast<int64_t>(qi_c - ds_i) * 32;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        uint4* ptr = reinterpret_cast<uint4*>(qtile + (c >> 3) * HALF + sw128_off(r, c & 7));
+        uint4 x = *ptr;
+        const float4 cs0 = __ldg(tab + 2 * c), cs1 = __ldg(tab + 2 * c + 1);
+        x.x = rope_rotate_pair(x.x, cs0.x, cs0.y);
+        x.y = rope_rotate_pair(x.y, cs0.z, cs0.w);
+        x.z = rope_rotate_pair(x.z, cs1.x, cs1.y);
+        x.w = rope_rotate_pair(x.w, cs1.z, cs1.w);
+        *ptr = x;
+      }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(bar(B_Q_READY + s));
+
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY;  // reference max, in log2 units of the scaled score
+    float l = 0.f;
+    for (int j = 0; ok && j < n_kv; ++j) {
+      const int kb = (kv_t0 + j) * BN;
+      if (!mbar_wait(bar(B_S_READY + s), j & 1, wc)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+      tc_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(B_S_FREE + s));
+
+      float sv[128];
+#pragma unroll
+      for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c]);
+      if (kb + BN - 1 > q0 || kb < ds_last) {
+        const int lo = ds_i - kb, hi = qi_c - kb;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) sv[c] = (c < lo || c > hi) ? -INFINITY : sv[c];
+      }
+      float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+#pragma unroll
+      for (int c = 4; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, sv[c]);
+        mx1 = fmaxf(mx1, sv[c + 1]);
+        mx2 = fmaxf(mx2, sv[c + 2]);
+        mx3 = fmaxf(mx3, sv[c + 3]);
+      }
+      const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const float m_new = fmaxf(m, mt);
+      const bool resc = m_new > m + kRescaleLog2;
+      float alpha = 1.f;
+      if (resc) {
+        alpha = ex2_approx(m - m_new);
+        m = m_new;
+      }
+      const float neg_m = (m == -INFINITY) ? 0.f : -m;
+      uint32_t pk[64];
+      float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 128; c += 2) {
+        const float p0 = ex2_approx(fmaf(sv[c], sl2, neg_m));
+        const float p1 = ex2_approx(fmaf(sv[c + 1], sl2, neg_m));
+        rs0 += p0;
+        rs1 += p1;
+        pk[c >> 1] = pack_bf16x2(p0, p1);
+      }
+      l = l * alpha + (rs0 + rs1);
+
+      if (j > 0) {
+        if (!mbar_wait(bar(B_PV_DONE + s), (j - 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t o[32];
+            tmem_ld32(tO + ch * 32, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+            tmem_st32(tO + ch * 32, o);
+          }
+          tc_wait_st();
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        uint4 w;
+        w.x = pk[4 * c];
+        w.y = pk[4 * c + 1];
+        w.z = pk[4 * c + 2];
+        w.w = pk[4 * c + 3];
+        *reinterpret_cast<uint4*>(ptile + (c >> 3) * HALF + sw128_off(r, c & 7)) = w;
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(B_P_READY + s));
+    }
+
+    // ---- epilogue: O / l -> bf16 -> Q tile buffer -> TMA store
+    if (ok) ok = mbar_wait(bar(B_PV_DONE + s), (n_kv - 1) & 1, wc);
+    tc_fence_after();
+    if (ok) {
+      const float inv_l = 1.f / l;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t o[32];
+        tmem_ld32(tO + ch * 32, o);
+        tc_wait_ld();
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(o[8 * c4 + 0]) * inv_l, __uint_as_float(o[8 * c4 + 1]) * inv_l);
+          w.y = pack_bf16x2(__uint_as_float(o[8 * c4 + 2]) * inv_l, __uint_as_float(o[8 * c4 + 3]) * inv_l);
+          w.z = pack_bf16x2(__uint_as_float(o[8 * c4 + 4]) * inv_l, __uint_as_float(o[8 * c4 + 5]) * inv_l);
+          w.w = pack_bf16x2(__uint_as_float(o[8 * c4 + 6]) * inv_l, __uint_as_float(o[8 * c4 + 7]) * inv_l);
+          const int d = ch * 32 + c4 * 8;
+          *reinterpret_cast<uint4*>(qtile + (d >> 6) * HALF + sw128_off(r, (d & 63) >> 3)) = w;
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    mbar_arrive(bar(B_O_STAGED + s));
+    if (r == 0 && ok && mbar_wait(bar(B_O_STAGED + s), 0, wc)) {
+      tma_store_4d(&tm_o, sbase + OFF_Q + s * TILE, 0, h0 + s, q0, b);
+      tma_store_4d(&tm_o, sbase + OFF_Q + s * TILE + HALF, 64, h0 + s, q0, b);
+      tma_store_commit();
+      tma_store_wait0();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace pfx
+}  // namespace la

@@ -1,0 +1,107 @@
+// rope.cuh -- RoPE cos/sin table, per-token document layout, and the K
+// rotation pass that feeds the tensor-core prefill.
+//
+// RoPE ("Llama 3.1 Architecture: Dense Scaling to 405B and 128K Context",
+// "Context Expansion", "High Base Frequency"): theta_k = base^(-2k/D),
+// k in [0, D/2 - 1]; the pair (x_2k, x_2k+1) of a token at position p turns by
+// p * theta_k (RoFormer rotation). Cross-document mask ("The Llama 3 Herd of
+// Models", architecture chapter): positions restart at each document.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace la {
+
+// tab[p * (D/2) + k] = (cos(p * theta_k), sin(p * theta_k)) for p < maxpos.
+// The angle is formed and reduced in float64 and only the result is rounded
+// to float32: a float32 product p * theta_k would be off by ~4e-3 rad at
+// p ~ 1.3e5.
+__global__ void rope_table_kernel(float2* __restrict__ tab, int maxpos, int D, double base) {
+  const int half = D / 2;
+  const int64_t n = static_cast<int64_t>(maxpos) * half;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int p = static_cast<int>(i / half), k = static_cast<int>(i % half);
+    const double freq = pow(base, -2.0 * static_cast<double>(k) / static_cast<double>(D));
+    double s, c;
+    sincos(static_cast<double>(p) * freq, &s, &c);
+    tab[i] = make_float2(static_cast<float>(c), static_cast<float>(s));
+  }
+}
+
+// Per-token row-local document start from doc_offsets (cumulative starts in
+// flattened B*S coordinates, ending with the sentinel B*S). One block: thread 0
+// walks and validates the offsets (their count is implicit), then every thread
+// binary-searches its tokens. Malformed offsets raise
+// LLAMA_ATTN_DEVERR_DOC_OFFSETS and every row is treated as one document, so
+// all later indexing stays in bounds.
+__global__ void doc_prep_kernel(const int32_t* __restrict__ offs, int B, int S,
+                                int32_t* __restrict__ doc_start) {
+  __shared__ int s_ndocs;
+  const int64_t total = static_cast<int64_t>(B) * S;
+  if (threadIdx.x == 0) {
+    int n = -1;
+    if (offs[0] == 0) {
+      int64_t prev = 0;
+      for (int64_t d = 1; d <= total; ++d) {
+        const int64_t o = offs[d];
+        if (o <= prev || o > total || (prev / S) != ((o - 1) / S)) break;
+        prev = o;
+        if (o == total) {
+          n = static_cast<int>(d);
+          break;
+        }
+      }
+    }
+    if (n < 0) raise_error(LLAMA_ATTN_DEVERR_DOC_OFFSETS);
+    s_ndocs = n;
+  }
+  __syncthreads();
+  const int n = s_ndocs;
+  for (int64_t t = threadIdx.x; t < total; t += blockDim.x) {
+    const int64_t row_start = (t / S) * S;
+    int32_t ds = 0;
+    if (n > 0) {
+      int lo = 0, hi = n - 1;  // largest d with offs[d] <= t
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (offs[mid] <= t) lo = mid; else hi = mid - 1;
+      }
+      ds = static_cast<int32_t>(offs[lo] - row_start);
+    }
+    doc_start[t] = ds;
+  }
+}
+
+// Rotate one bf16 pair (low half = element 2k, high half = element 2k+1).
+__device__ __forceinline__ uint32_t rope_rotate_pair(uint32_t xv, float c, float s) {
+  const float2 x = unpack_bf16x2(xv);
+  return pack_bf16x2(x.x * c - x.y * s, x.x * s + x.y * c);
+}
+
+// y = RoPE(x) for x [B, S, H, 128] bf16 at each token's document position.
+// One thread per 16-byte vector (4 pairs); the table row of the token is read
+// as float4s (2 pairs each).
+__global__ void rope_rotate_rows_bf16_kernel(const uint4* __restrict__ x, uint4* __restrict__ y,
+                                             const float4* __restrict__ tab,
+                                             const int32_t* __restrict__ doc_start, int S, int H,
+                                             int64_t n_vec) {
+  constexpr int kVecPerRow = 16;  // 128 bf16 per head row
+  for (int64_t v = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; v < n_vec;
+       v += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = v / (static_cast<int64_t>(H) * kVecPerRow);
+    const int c = static_cast<int>(v % kVecPerRow);
+    const int i = static_cast<int>(t % S);
+    const int pos = i - (doc_start ? doc_start[t] : 0);
+    const float4* tp = tab + static_cast<int64_t>(pos) * 32 + c * 2;
+    const float4 cs0 = __ldg(tp), cs1 = __ldg(tp + 1);
+    uint4 xv = x[v];
+    xv.x = rope_rotate_pair(xv.x, cs0.x, cs0.y);
+    xv.y = rope_rotate_pair(xv.y, cs0.z, cs0.w);
+    xv.z = rope_rotate_pair(xv.z, cs1.x, cs1.y);
+    xv.w = rope_rotate_pair(xv.w, cs1.z, cs1.w);
+    y[v] = xv;
+  }
+}
+
+}  // namespace la

@@ -1,0 +1,161 @@
+/*
+ * llama_attn.h -- C ABI of the B200 (sm_100a) attention library for the dense
+ * Llama 3 / 3.1 decoder: grouped-query causal attention with rotary position
+ * embeddings and the cross-document mask, as a prefill over packed sequences
+ * and as a single-token decode against a KV cache.
+ *
+ * What the calls compute (the pages' statement of the method):
+ *   - RoPE frequencies theta_k = rope_theta^(-2k/D), k in [0, D/2 - 1]
+ *     ("Llama 3.1 Architecture: Dense Scaling to 405B and 128K Context",
+ *     "Context Expansion", "High Base Frequency"); base 500,000 for Llama 3
+ *     (same subsection; "The Llama 3 Herd of Models", architecture chapter).
+ *     The rotation turns adjacent pairs (x_2k, x_2k+1) by p * theta_k
+ *     (RoFormer, cited on the first page), p = the token's position.
+ *   - Grouped-query attention: query head h reads KV head h / (Hq / Hkv)
+ *     ("How Meta's Llama 3.1 405B Architecture Actually Works", GQA
+ *     paragraph; 128 query heads over 8 KV heads on the 405B chart).
+ *   - Causal attention with the cross-document mask ("The Llama 3 Herd of
+ *     Models", architecture chapter): key j is visible to query i iff both are
+ *     in the same batch row and the same document and j <= i. Positions
+ *     restart at 0 at each document start. Scores are scaled by 1/sqrt(D).
+ *   - Decode: the KV cache of GQA ("How Meta's Llama 3.1 405B ...", GQA
+ *     paragraph: the KV cache used while decoding) holds keys already rotated
+ *     at their positions; the new query is rotated at position len.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers to contiguous memory, owned by
+ *     the caller. bf16 tensors are passed as raw 16-bit patterns.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream) and do
+ *     not synchronise the host, except that the first use of a (device, theta,
+ *     D) RoPE table, or a request that outgrows a cached table or scratch
+ *     buffer, allocates device memory (cudaMalloc) before enqueueing work.
+ *   - Arguments are checked on the host before anything is launched; a
+ *     failed check returns a negative status and launches nothing.
+ *   - The library keeps per-device caches (RoPE tables, scratch); calls from
+ *     several host threads at once are not supported.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef LLAMA_ATTN_H
+#define LLAMA_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same underlying type as the CUDA runtime's cudaStream_t. */
+typedef struct CUstream_st *cudaStream_t;
+
+/* Raw bf16 bit pattern (1 sign, 8 exponent, 7 mantissa bits). */
+typedef uint16_t llama_attn_bf16;
+
+typedef enum {
+  LLAMA_ATTN_OK = 0,
+  LLAMA_ATTN_ERR_INVALID_ARG = -1, /* null pointer, non-positive size, Hq % Hkv != 0, ... */
+  LLAMA_ATTN_ERR_UNSUPPORTED = -2, /* a shape the kernels do not implement (e.g. D != 128 on bf16) */
+  LLAMA_ATTN_ERR_WORKSPACE = -3,   /* decode workspace missing or too small */
+  LLAMA_ATTN_ERR_CUDA = -4,        /* a CUDA runtime/driver call or a launch failed */
+  LLAMA_ATTN_ERR_DEVICE = -5       /* a kernel reported an error word (see get_device_error) */
+} llama_attn_status;
+
+/*
+ * Prefill, bf16 in / bf16 out, fp32 accumulation (tcgen05 tensor cores).
+ *
+ *   q   [B, S, Hq,  D]  un-rotated queries
+ *   k   [B, S, Hkv, D]  un-rotated keys
+ *   v   [B, S, Hkv, D]  values
+ *   out [B, S, Hq,  D]  result (must not alias q, k or v)
+ *   doc_offsets: NULL (each batch row is one document), or a device int32
+ *     array of document starts in flattened B*S token coordinates:
+ *     0 = o_0 < o_1 < ... < o_n = B*S, ending with the sentinel B*S; no
+ *     document crosses a batch-row boundary. Its length is implicit (it is
+ *     read up to the sentinel). A malformed array is detected on the device:
+ *     the output is then unspecified and the device error word is set to
+ *     LLAMA_ATTN_DEVERR_DOC_OFFSETS.
+ *   B, S >= 1; Hq, Hkv >= 1 with Hq % Hkv == 0; D == 128; rope_theta > 0.
+ *   Scratch: the call keeps a library-owned rotated copy of k (B*S*Hkv*D bf16)
+ *   and per-token document data, grown on demand.
+ */
+int llama_attn_prefill(const llama_attn_bf16 *q, const llama_attn_bf16 *k,
+                       const llama_attn_bf16 *v, llama_attn_bf16 *out,
+                       const int32_t *doc_offsets, int B, int S, int Hq, int Hkv, int D,
+                       float rope_theta, cudaStream_t stream);
+
+/*
+ * Prefill in true fp32 arithmetic on CUDA cores (FFMA, accurate expf), same
+ * semantics and layouts as llama_attn_prefill with float tensors.
+ * D even, 2 <= D <= 128.
+ */
+int llama_attn_prefill_f32(const float *q, const float *k, const float *v, float *out,
+                           const int32_t *doc_offsets, int B, int S, int Hq, int Hkv, int D,
+                           float rope_theta, cudaStream_t stream);
+
+/*
+ * Bytes of device workspace llama_attn_decode needs for these sizes (split-KV
+ * partial outputs and log-sum-exps). Returns 0 for invalid sizes.
+ */
+size_t llama_attn_decode_workspace_size(int B, int Hq, int Lmax, int D);
+
+/*
+ * Single-token decode against a KV cache, bf16 in / bf16 out, fp32 math.
+ *
+ *   q          [B, Hq, D]          un-rotated query of the new token
+ *   kcache     [B, Hkv, Lmax, D]   keys, row n already rotated at position n
+ *   vcache     [B, Hkv, Lmax, D]   values
+ *   cache_lens [B] int32, device   valid rows per sequence, 0 <= len <= Lmax
+ *   out        [B, Hq, D]
+ *   The query of sequence b is rotated at position cache_lens[b] and attends
+ *   to cache rows 0 .. cache_lens[b]-1 (the new token's own key/value are the
+ *   caller's to append). Rows at or past cache_lens[b] are never used, so they
+ *   may hold anything. cache_lens[b] == 0 gives out = 0. A length outside
+ *   [0, Lmax] sets LLAMA_ATTN_DEVERR_CACHE_LEN and that sequence's output is 0.
+ *   D == 128; Hq % Hkv == 0 and Hq / Hkv <= 16; Lmax >= 1.
+ *   workspace: device memory of at least
+ *   llama_attn_decode_workspace_size(B, Hq, Lmax, D) bytes, 16-byte aligned,
+ *   owned by the caller; its contents need no initialisation.
+ */
+int llama_attn_decode(const llama_attn_bf16 *q, const llama_attn_bf16 *kcache,
+                      const llama_attn_bf16 *vcache, const int32_t *cache_lens,
+                      llama_attn_bf16 *out, int B, int Hq, int Hkv, int D, int Lmax,
+                      float rope_theta, void *workspace, size_t workspace_bytes,
+                      cudaStream_t stream);
+
+/* Static, human-readable text for a status code. Never NULL. */
+const char *llama_attn_status_string(int status);
+
+/* Device error word bits (kernels OR them in; they never trap). */
+#define LLAMA_ATTN_DEVERR_TIMEOUT 0x1     /* a bounded wait on a barrier gave up */
+#define LLAMA_ATTN_DEVERR_DOC_OFFSETS 0x2 /* malformed doc_offsets */
+#define LLAMA_ATTN_DEVERR_CACHE_LEN 0x4   /* cache_lens[b] outside [0, Lmax] */
+
+/*
+ * Waits for `stream`, then returns and clears the current device's error word
+ * (0 = no error). Returns a negative llama_attn_status if the CUDA calls
+ * themselves fail.
+ */
+int llama_attn_get_device_error(cudaStream_t stream);
+
+/*
+ * Benchmark instrumentation (host side, current device only).
+ * llama_attn_profile_begin() starts a session: each later prefill / decode call
+ * records a CUDA event pair on its stream around its main kernel (prefill: the
+ * attention kernel; decode: the split-KV kernel) and every kernel the library
+ * launches is counted. llama_attn_profile_end() waits for the recorded events,
+ * writes the summed main-kernel time in milliseconds, the number of timed main
+ * kernels and the number of kernels launched, and ends the session. At most
+ * 4096 main kernels are timed per session; later ones are counted only.
+ * Returns LLAMA_ATTN_OK or a negative status. Any output pointer may be NULL.
+ */
+int llama_attn_profile_begin(void);
+int llama_attn_profile_end(double *main_kernel_ms, int *main_kernels_timed, int *kernels_launched);
+
+/* Library version, as MAJOR * 10000 + MINOR * 100 + PATCH. */
+int llama_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLAMA_ATTN_H */

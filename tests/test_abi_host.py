@@ -1,0 +1,114 @@
+"""CPU tests of the C-ABI library: it loads, exports every function the header
+declares, and rejects bad arguments on the host before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gqa_attention_rope_b200 as la
+from gqa_attention_rope_b200 import build as labuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, INVALID, UNSUPPORTED, WORKSPACE = 0, -1, -2, -3
+
+
+@pytest.fixture(scope="module")
+def lib():
+    labuild.build()
+    return la.load_library()
+
+
+def header_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for fn in os.listdir(inc):
+        if fn.endswith(".h"):
+            src = open(os.path.join(inc, fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"\b(llama_attn_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_symbols_exported(lib):
+    names = header_functions()
+    assert "llama_attn_prefill" in names and "llama_attn_decode" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    assert set(la.EXPORTED) <= set(names)
+
+
+def test_status_strings_and_version(lib):
+    for st in (0, -1, -2, -3, -4, -5, 7):
+        s = lib.llama_attn_status_string(st)
+        assert isinstance(s, bytes) and len(s) > 0
+    assert lib.llama_attn_version() >= 100
+
+
+def test_workspace_size(lib):
+    f = lib.llama_attn_decode_workspace_size
+    assert f(0, 64, 32768, 128) == 0
+    assert f(64, 64, 32768, 64) == 0
+    n = f(64, 64, 32768, 128)
+    nchunk = 32
+    assert n >= 64 * 64 * nchunk * 129 * 4 and n % 256 == 0
+    assert f(1, 1, 1, 128) >= 129 * 4
+
+
+FAKE = ctypes.c_void_p(4096)  # never dereferenced: every case below fails validation first
+
+
+@pytest.mark.parametrize("args,expect", [
+    # q, k, v, out, offs, B, S, Hq, Hkv, D, theta
+    ((None, FAKE, FAKE, FAKE, None, 1, 128, 8, 2, 128, 5e5), INVALID),
+    ((FAKE, FAKE, FAKE, None, None, 1, 128, 8, 2, 128, 5e5), INVALID),
+    ((FAKE, FAKE, FAKE, FAKE, None, 0, 128, 8, 2, 128, 5e5), INVALID),
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 0, 8, 2, 128, 5e5), INVALID),
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 128, 8, 3, 128, 5e5), INVALID),
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 128, 8, 2, 128, -1.0), INVALID),
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 128, 8, 2, 64, 5e5), UNSUPPORTED),
+    ((ctypes.c_void_p(4098), FAKE, FAKE, FAKE, None, 1, 128, 8, 2, 128, 5e5), INVALID),
+])
+def test_prefill_rejects(lib, args, expect):
+    assert lib.llama_attn_prefill(*args, None) == expect
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((None, FAKE, FAKE, FAKE, None, 1, 128, 8, 2, 64, 5e5), INVALID),
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 128, 8, 2, 63, 5e5), UNSUPPORTED),
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 128, 8, 2, 256, 5e5), UNSUPPORTED),
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 128, 8, 0, 64, 5e5), INVALID),
+])
+def test_prefill_f32_rejects(lib, args, expect):
+    assert lib.llama_attn_prefill_f32(*args, None) == expect
+
+
+def test_decode_rejects(lib):
+    f = lib.llama_attn_decode
+    big = 1 << 40
+    # q, kc, vc, lens, out, B, Hq, Hkv, D, Lmax, theta, ws, ws_bytes
+    assert f(None, FAKE, FAKE, FAKE, FAKE, 2, 16, 2, 128, 64, 5e5, FAKE, big, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 16, 3, 128, 64, 5e5, FAKE, big, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 16, 2, 64, 64, 5e5, FAKE, big, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 64, 2, 128, 64, 5e5, FAKE, big, None) == UNSUPPORTED  # G = 32
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 16, 2, 128, 0, 5e5, FAKE, big, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 16, 2, 128, 64, 5e5, None, big, None) == WORKSPACE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 16, 2, 128, 64, 5e5, FAKE, 16, None) == WORKSPACE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 16, 2, 128, 64, 5e5, ctypes.c_void_p(4100), big, None) == WORKSPACE
+
+
+def test_python_binding_fails_loudly_without_library(tmp_path):
+    with pytest.raises(RuntimeError, match="not found"):
+        la.load_library(str(tmp_path / "missing.so"))
+
+
+def test_shard_units_partition():
+    for n in (0, 1, 7, 32, 100):
+        for w in (1, 2, 3, 8):
+            seen = []
+            for r in range(w):
+                rg = la.shard_units(n, w, r)
+                seen += list(rg)
+                assert len(rg) in (n // w, n // w + 1)
+            assert seen == list(range(n))
