@@ -22,7 +22,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -49,51 +48,64 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle sampling while the timed region runs."""
+    """SM clock and clock-event reasons sampled every 5 ms (NVML, in a thread)
+    while the timed region runs; falls back to nvidia-smi."""
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.path = None
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.samples = []
+        self.reasons = set()
+        self._stop = None
+        self._thread = None
+        self.max_mhz = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            bus = torch.cuda.get_device_properties(self.cuda_index).pci_bus_id
+            return pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode() if isinstance(bus, str) else bus)
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
     def start(self):
-        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{self.index}.csv")
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        import threading
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            import pynvml
+            h = self._handle()
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
         except Exception:
-            self.proc = None
+            self._thread = None
+            return
+        self._stop = threading.Event()
+
+        def run():
+            get_r = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                    bits = get_r(h)
+                    for b, n in self.REASONS.items():
+                        if bits & b:
+                            self.reasons.add(n)
+                except Exception:
+                    pass
+                self._stop.wait(0.005)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                smax.append(float(f[2]))
-            except ValueError:
-                continue
-            for n, val in zip(names, f[5:9]):
-                if val.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if self._thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"], "samples": 0}
+        self._stop.set()
+        self._thread.join()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 def dist_setup(n_gpus: int):
@@ -224,7 +236,7 @@ def run_ours(args, w):
     if la.llama_attn_get_device_error() != 0:
         raise RuntimeError("device error word set during warm-up")
 
-    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    clocks = ClockSampler(local)
     clocks.start()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier(world)
@@ -314,6 +326,9 @@ def run_ours(args, w):
 
 def run_decode(args, la, dev, world, rank, hbm_peak, peak_kind):
     w = W.DECODE_70B
+    nseq = args.decode_seqs
+    name = w.name if nseq == w.B else w.name.replace(f"B{w.B}_", f"B{nseq}_")
+    w = W.DecodeWorkload(name, w.seed, nseq, w.Hq, w.Hkv, w.D, w.Lmax, w.len_range)
     wr = W.DecodeWorkload(w.name, w.seed + 1000 * rank, w.B, w.Hq, w.Hkv, w.D, w.Lmax, w.len_range)
     inp = W.make_decode_inputs(wr, poison=True)
     q, kc, vc, lens = (inp[n].to(dev) for n in ("q", "kcache", "vcache", "cache_lens"))
@@ -359,12 +374,18 @@ def run_decode(args, la, dev, world, rank, hbm_peak, peak_kind):
 
 
 def load_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if one matches."""
+    """DRAM bytes per launch from the committed ncu record, or None when there is
+    no record for this kernel and workload or the kernel source has changed
+    since the counters were taken."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            t = json.load(f)
-        return t[kernel][workload]
+            rec = json.load(f)[kernel][workload]
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            if hashlib.sha1(f.read()).hexdigest() != rec["source_sha1"]:
+                return None
+        return rec["bytes"]
     except Exception:
         return None
 
@@ -372,12 +393,14 @@ def load_traffic(kernel: str, workload: str):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=W.PACKED_8B.name, choices=[n for n, x in W.WORKLOADS.items()
                                                                       if isinstance(x, W.PrefillWorkload)])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-seqs", type=int, default=W.DECODE_70B.B,
+                    help="sequences in the decode batch (64 = the 70B-shaped workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()

@@ -131,7 +131,7 @@ def custom_prefill(seed: int, B: int, S: int, Hq: int, Hkv: int, D: int, dtype: 
     return PrefillWorkload(name, seed, B, S, Hq, Hkv, D, dtype, doc_range, rope_theta)
 
 
-def make_decode_inputs(w: DecodeWorkload, poison: bool = True):
+def make_decode_inputs(w: DecodeWorkload, poison: bool = True, lens=None):
     """Returns dict(q, kcache, vcache, cache_lens) as CPU tensors.
 
     q is [B, Hq, D]; kcache and vcache are [B, Hkv, Lmax, D] and hold keys that
@@ -139,10 +139,12 @@ def make_decode_inputs(w: DecodeWorkload, poison: bool = True):
     draw is used directly as those rotated keys: a rotation maps an iid
     Gaussian vector to an iid Gaussian vector, so the distribution is the one
     the workload names. Rows at or past cache_lens[b] are NaN when ``poison``.
+    ``lens`` (optional) replaces the drawn cache lengths.
     """
     gen = torch.Generator().manual_seed(w.seed)
-    lens = torch.randint(w.len_range[0], w.len_range[1] + 1, (w.B,), generator=gen,
-                         dtype=torch.int64).to(torch.int32)
+    drawn = torch.randint(w.len_range[0], w.len_range[1] + 1, (w.B,), generator=gen,
+                          dtype=torch.int64).to(torch.int32)
+    lens = drawn if lens is None else torch.as_tensor(lens, dtype=torch.int32)
     q = _randn(gen, (w.B, w.Hq, w.D), w.dtype)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     fill = float("nan") if poison else 0.0

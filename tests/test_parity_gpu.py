@@ -136,13 +136,10 @@ DECODE_CASES = [
 @pytest.mark.parametrize("B,Hq,Hkv,Lmax,lens", DECODE_CASES)
 def test_decode_small(B, Hq, Hkv, Lmax, lens):
     w = W.custom_decode(21 + B, B, Hq, Hkv, 128, Lmax, (1, Lmax))
-    inp = W.make_decode_inputs(w, poison=True)
-    inp["cache_lens"] = torch.tensor(lens, dtype=torch.int32)
+    inp = W.make_decode_inputs(w, poison=True, lens=lens)
     out = la.llama_attn_decode(*(to_dev(inp[n]) for n in ("q", "kcache", "vcache", "cache_lens")))
     torch.cuda.synchronize()
-    kc = torch.nan_to_num(inp["kcache"], nan=0.0)
-    vc = torch.nan_to_num(inp["vcache"], nan=0.0)
-    ref = O.decode(inp["q"], kc, vc, inp["cache_lens"])
+    ref = O.decode(inp["q"], inp["kcache"], inp["vcache"], inp["cache_lens"])
     got = out.float().cpu().numpy()
     report(got, ref, TOL_BF16, f"decode lens={lens}")
     for b, n in enumerate(lens):
