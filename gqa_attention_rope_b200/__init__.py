@@ -26,6 +26,7 @@ EXPORTED = (
     "llama_attn_version",
     "llama_attn_profile_begin",
     "llama_attn_profile_end",
+    "llama_attn_decode_noalloc",
 )
 
 DEVERR_TIMEOUT = 0x1
@@ -68,6 +69,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.llama_attn_profile_begin.restype = I
     lib.llama_attn_profile_end.argtypes = [P, P, P]
     lib.llama_attn_profile_end.restype = I
+    lib.llama_attn_decode_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P]
+    lib.llama_attn_decode_noalloc.restype = I
     return lib
 
 
@@ -191,6 +194,24 @@ def llama_attn_decode(q, kcache, vcache, cache_lens, out=None, workspace=None, r
                                  Lmax, float(rope_theta), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                  _stream(stream))
     _check("llama_attn_decode", st)
+    return out
+
+
+def llama_attn_decode_noalloc(q, kcache, vcache, cache_lens, out, rope_theta: float = 500000.0, stream=None):
+    """llama_attn_decode without a workspace or any device allocation, for
+    callers that cannot allocate: the partials go to a fixed 72 MiB array in the
+    library. ``out`` must be supplied by the caller (nothing is allocated here)."""
+    import torch
+    _require(q.dim() == 3 and kcache.dim() == 4 and vcache.shape == kcache.shape, "bad shapes")
+    for t in (q, kcache, vcache, out):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "bf16 contiguous CUDA tensors expected")
+    _require(cache_lens.is_cuda and cache_lens.dtype == torch.int32, "cache_lens: int32 CUDA tensor")
+    B, Hq, D = q.shape
+    Hkv, Lmax = kcache.shape[1], kcache.shape[2]
+    _require(out.shape == q.shape and cache_lens.numel() == B, "bad shapes")
+    st = lib().llama_attn_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(cache_lens), _ptr(out), B, Hq,
+                                         Hkv, D, Lmax, float(rope_theta), _stream(stream))
+    _check("llama_attn_decode_noalloc", st)
     return out
 
 

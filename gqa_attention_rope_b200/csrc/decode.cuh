@@ -35,6 +35,9 @@ constexpr uint32_t KHALF = ROWS * 128;      // 64 rows x 64 bf16 = 8 KB
 constexpr uint32_t STAGE = 4 * KHALF;       // K (2 halves) + V (2 halves)
 constexpr uint32_t OFF_BAR = NSTAGE * STAGE;
 constexpr uint32_t SMEM_ALLOC = OFF_BAR + 64 + 1024;
+// The variant that computes its own (cos, sin) row keeps it after the barriers.
+constexpr uint32_t OFF_SELF_TABLE = OFF_BAR + 64;
+constexpr uint32_t SMEM_ALLOC_SELF_TABLE = SMEM_ALLOC + 64 * 8;
 static_assert(NCW * (2 * 16 + 16 * 128) * 4 <= OFF_BAR, "combine scratch fits in the ring");
 
 struct Params {
@@ -46,10 +49,16 @@ struct Params {
   float* part_o;             // [B, Hq, nchunk, 128]
   float* part_lse;           // [B, Hq, nchunk]
   unsigned int epoch;        // launch id for bounded-wait abort propagation
+  double rope_theta;         // used only when the kernel forms its own (cos, sin) row
 };
 
 __device__ __forceinline__ int valid_len(int len, int Lmax) { return (len < 0 || len > Lmax) ? 0 : len; }
 
+// kSelfTable = false: (cos, sin) at position len come from the cached table
+// p.rope_tab. kSelfTable = true: the CTA forms that one row itself (float64
+// angle, same formula as rope_table_kernel) in shared memory, so no table needs
+// to be allocated.
+template <bool kSelfTable>
 __global__ void __launch_bounds__(NTHREADS, 2)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const Params p) {
@@ -78,6 +87,15 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     fence_mbar_init();
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
+  }
+  if constexpr (kSelfTable) {
+    if (threadIdx.x < 64) {
+      const double freq = pow(p.rope_theta, -2.0 * static_cast<double>(threadIdx.x) / 128.0);
+      double sn, cs;
+      sincos(static_cast<double>(len) * freq, &sn, &cs);
+      reinterpret_cast<float2*>(smem + OFF_SELF_TABLE)[threadIdx.x] =
+          make_float2(static_cast<float>(cs), static_cast<float>(sn));
+    }
   }
   __syncthreads();
 
@@ -108,7 +126,8 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   // A fragments of the rotated query: rows = heads of the group (row >= G is zero).
   uint32_t qa[8][4];
   {
-    const float4* tab = p.rope_tab + static_cast<int64_t>(len) * 32;
+    const float4* tab = kSelfTable ? reinterpret_cast<const float4*>(smem + OFF_SELF_TABLE)
+                                   : p.rope_tab + static_cast<int64_t>(len) * 32;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
 #pragma unroll
@@ -119,7 +138,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         if (row < G) {
           const uint32_t x = *reinterpret_cast<const uint32_t*>(
               p.q + (static_cast<int64_t>(b) * p.Hq + gk * G + row) * 128 + d);
-          const float4 cs = __ldg(tab + (d >> 2));
+          const float4 cs = kSelfTable ? tab[d >> 2] : __ldg(tab + (d >> 2));
           const float cc = (d & 2) ? cs.z : cs.x, ss = (d & 2) ? cs.w : cs.y;
           val = rope_rotate_pair(x, cc, ss);
         }

@@ -216,6 +216,19 @@ int check_prefill_common(const void* q, const void* k, const void* v, const void
 
 }  // namespace
 
+// ---- scratch for llama_attn_decode_noalloc
+// A fixed device array replaces the caller's decode workspace for callers that
+// cannot allocate device memory. Every device that loads this library holds it
+// until the process exits. In host code the name is only a host-side handle:
+// its device address comes from cudaGetSymbolAddress, once per device.
+constexpr size_t kNoAllocScratchBytes = size_t(72) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+void* g_noalloc_scratch_addr[kMaxDevices];
+bool g_noalloc_attr_set[kMaxDevices];
+}  // namespace
+
 extern "C" {
 
 int llama_attn_version(void) { return LLAMA_ATTN_VERSION; }
@@ -424,21 +437,75 @@ int llama_attn_decode(const llama_attn_bf16* q, const llama_attn_bf16* kcache, c
   p.rope_tab = reinterpret_cast<const float4*>(tab);
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   p.epoch = next_epoch();
+  p.rope_theta = static_cast<double>(rope_theta);
   const size_t slots = static_cast<size_t>(B) * Hq * p.nchunk;
   p.part_o = static_cast<float*>(workspace);
   p.part_lse = p.part_o + slots * 128;
   if (!dc.decode_attr_set) {
-    LA_CUDA(cudaFuncSetAttribute(la::dec::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    LA_CUDA(cudaFuncSetAttribute(la::dec::decode_split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  la::dec::SMEM_ALLOC));
     dc.decode_attr_set = true;
   }
   const dim3 grid(p.nchunk, Hkv, B);
   prof_count(2);
   const int pair = prof_before(stream);
-  la::dec::decode_split_kernel<<<grid, la::dec::NTHREADS, la::dec::SMEM_ALLOC, stream>>>(tk, tv, p);
+  la::dec::decode_split_kernel<false><<<grid, la::dec::NTHREADS, la::dec::SMEM_ALLOC, stream>>>(tk, tv, p);
   const cudaError_t e = cudaGetLastError();
   prof_after(pair, stream);
   if (e != cudaSuccess) return LLAMA_ATTN_ERR_CUDA;
+  la::dec::decode_combine_kernel<<<B * Hq, 128, 0, stream>>>(p.part_o, p.part_lse, cache_lens, out, Hq, Lmax,
+                                                            p.nchunk);
+  return cuda_status(cudaGetLastError());
+}
+
+int llama_attn_decode_noalloc(const llama_attn_bf16* q, const llama_attn_bf16* kcache,
+                              const llama_attn_bf16* vcache, const int32_t* cache_lens, llama_attn_bf16* out, int B,
+                              int Hq, int Hkv, int D, int Lmax, float rope_theta, cudaStream_t stream) {
+  if (!q || !kcache || !vcache || !cache_lens || !out) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lmax <= 0 || Hq % Hkv != 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.f) || !std::isfinite(rope_theta)) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (D != 128 || Hq / Hkv > 16) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535 || B * Hq > INT32_MAX / 2) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * Hkv * Lmax >= INT32_MAX) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(kcache) || !aligned16(vcache) || !aligned16(q) || !aligned16(out)) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (llama_attn_decode_workspace_size(B, Hq, Lmax, D) > kNoAllocScratchBytes) return LLAMA_ATTN_ERR_WORKSPACE;
+  int dev, st;
+  if ((st = current_device(&dev))) return st;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_noalloc_scratch_addr[dev] == nullptr) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || addr == nullptr) return LLAMA_ATTN_ERR_CUDA;
+    g_noalloc_scratch_addr[dev] = addr;
+  }
+  if (!g_noalloc_attr_set[dev]) {
+    LA_CUDA(cudaFuncSetAttribute(la::dec::decode_split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 la::dec::SMEM_ALLOC_SELF_TABLE));
+    g_noalloc_attr_set[dev] = true;
+  }
+  CUtensorMap tk, tv;
+  const int64_t rows = static_cast<int64_t>(B) * Hkv * Lmax;
+  if ((st = tmap_rows(&tk, kcache, rows))) return st;
+  if ((st = tmap_rows(&tv, vcache, rows))) return st;
+
+  la::dec::Params p;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.Lmax = Lmax;
+  p.nchunk = (Lmax + la::dec::CHUNK - 1) / la::dec::CHUNK;
+  p.lens = cache_lens;
+  p.q = q;
+  p.rope_tab = nullptr;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  p.epoch = next_epoch();
+  p.rope_theta = static_cast<double>(rope_theta);
+  const size_t slots = static_cast<size_t>(B) * Hq * p.nchunk;
+  p.part_o = static_cast<float*>(g_noalloc_scratch_addr[dev]);
+  p.part_lse = p.part_o + slots * 128;
+  const dim3 grid(p.nchunk, Hkv, B);
+  la::dec::decode_split_kernel<true><<<grid, la::dec::NTHREADS, la::dec::SMEM_ALLOC_SELF_TABLE, stream>>>(tk, tv, p);
+  LA_CUDA(cudaGetLastError());
   la::dec::decode_combine_kernel<<<B * Hq, 128, 0, stream>>>(p.part_o, p.part_lse, cache_lens, out, Hq, Lmax,
                                                             p.nchunk);
   return cuda_status(cudaGetLastError());

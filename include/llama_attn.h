@@ -122,6 +122,35 @@ int llama_attn_decode(const llama_attn_bf16 *q, const llama_attn_bf16 *kcache,
                       float rope_theta, void *workspace, size_t workspace_bytes,
                       cudaStream_t stream);
 
+/*
+ * llama_attn_decode without a caller-supplied workspace and without any
+ * device allocation, for callers that cannot allocate device memory: code
+ * that runs inside a CUDA graph capture, under an allocator that owns all of
+ * device memory, or in a host without access to cudaMalloc. Nothing on the
+ * pages corresponds to it; it exists only for such callers.
+ *
+ * Same arguments, layouts, results and error codes as llama_attn_decode, minus
+ * the workspace. The split-KV partials live in one fixed 72 MiB device array
+ * inside the library, which every device that loads the library holds until
+ * the process exits. A request needing more than that
+ * (llama_attn_decode_workspace_size(B, Hq, Lmax, D) > 72 MiB, i.e. more than
+ * 146,312 slots of B * Hq * ceil(Lmax / 1024)) is rejected with
+ * LLAMA_ATTN_ERR_WORKSPACE before anything is launched. The RoPE angle of the
+ * query is formed inside the kernel, so no table is allocated either.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and sets a kernel attribute; make that first call
+ * outside any stream capture. All calls share the one array and it keeps the
+ * last call's contents; nothing in it needs to start at zero, because every
+ * partial is written before it is read within a call. Calls whose kernels can
+ * overlap on the GPU (different streams, no ordering between them) race on
+ * the array: order them, e.g. on one stream.
+ */
+int llama_attn_decode_noalloc(const llama_attn_bf16 *q, const llama_attn_bf16 *kcache,
+                              const llama_attn_bf16 *vcache, const int32_t *cache_lens,
+                              llama_attn_bf16 *out, int B, int Hq, int Hkv, int D, int Lmax,
+                              float rope_theta, cudaStream_t stream);
+
 /* Static, human-readable text for a status code. Never NULL. */
 const char *llama_attn_status_string(int status);
 
