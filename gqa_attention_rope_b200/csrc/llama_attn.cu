@@ -34,6 +34,7 @@ struct DeviceCache {
   size_t krot_bytes = 0;
   int32_t* doc_start = nullptr;
   size_t doc_bytes = 0;
+  int* sched = nullptr;  // work-item counter of the persistent prefill kernel
   bool prefill_attr_set = false;
   bool decode_attr_set = false;
 };
@@ -338,6 +339,9 @@ int llama_attn_prefill(const llama_attn_bf16* q, const llama_attn_bf16* k, const
   p.rope_tab = reinterpret_cast<const float4*>(tab);
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
   p.epoch = next_epoch();
+  if (dc.sched == nullptr) LA_CUDA(cudaMalloc(&dc.sched, 256));
+  LA_CUDA(cudaMemsetAsync(dc.sched, 0, sizeof(int), stream));
+  p.sched = dc.sched;
   const int64_t items = static_cast<int64_t>(B) * p.n_qt * p.n_hp;
   if (items > INT32_MAX) return LLAMA_ATTN_ERR_UNSUPPORTED;
   if (!dc.prefill_attr_set) {
@@ -347,8 +351,10 @@ int llama_attn_prefill(const llama_attn_bf16* q, const llama_attn_bf16* k, const
   }
   prof_count(1);
   const int pair = prof_before(stream);
-  la::pfx::prefill_bf16_kernel<<<static_cast<int>(items), la::pfx::NTHREADS, la::pfx::SMEM_ALLOC, stream>>>(
-      tq, tk, tv, to, p);
+  int n_sm = 148;
+  if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
+  const int grid = static_cast<int>(items < n_sm ? items : n_sm);
+  la::pfx::prefill_bf16_kernel<<<grid, la::pfx::NTHREADS, la::pfx::SMEM_ALLOC, stream>>>(tq, tk, tv, to, p);
   const cudaError_t e = cudaGetLastError();
   prof_after(pair, stream);
   return cuda_status(e);

@@ -6,9 +6,14 @@
 //
 //   warp 0      TMA producer: Q tiles once, then K/V tiles through a 3-stage ring
 //               in the order the MMA warp consumes them (K0, K1, V0, K2, V1, ...).
-//   warp 1      TMEM owner and single-thread MMA issuer:
-//                 S_h = Q_h K_j^T   (M=128, N=128, K=128; accumulators in TMEM)
-//                 O_h += P_h V_j    (P from shared memory, V MN-major)
+//   warp 1      TMEM owner; one thread issues S_h = Q_h K_j^T (M=128, N=128,
+//               K=128; fp32 accumulators in TMEM)
+//   warp 2      one thread issues O_h += P_h V_j (P from shared memory, V MN-major).
+//               Two issuing threads: a tcgen05.mma issue blocks at the tensor
+//               rate and every barrier wait (~250+ cycles even when the phase
+//               has completed) would otherwise leave the tensor pipe idle; with
+//               S and PV issued from different threads one thread's waits
+//               overlap the other's MMAs.
 //   warps 4-7   softmax for head slot 0, warps 8-11 for slot 1: thread = query
 //               row = TMEM lane. Rotates its Q row in shared memory (RoPE at the
 //               row's document position), then per KV tile: S from TMEM ->
@@ -63,15 +68,19 @@ enum : int {
   B_P_READY = B_S_FREE + 2,
   B_PV_DONE = B_P_READY + 2,
   B_O_STAGED = B_PV_DONE + 2,
-  B_DRAIN = B_O_STAGED + 2,
+  B_O_READ = B_O_STAGED + 2,
+  B_Q_FREE = B_O_READ + 2,
+  B_DRAIN,
+  B_DRAIN_PV,
   N_BARS
 };
-static_assert(N_BARS * 8 + 8 <= 256, "barrier area");
+static_assert(N_BARS * 8 + 8 + 16 <= 256, "barrier area, TMEM address and item ring");
 
 struct Params {
   int B, S, Hq, Hkv, G, NH, n_qt, n_hp;
   const int32_t* doc_start;  // [B*S] row-local document start, or null (one document per row)
   const float4* rope_tab;    // (cos, sin) pairs, 64 per position, as float4 = 2 pairs
+  int* sched;                // work-item counter, zero at launch
   float scale_log2;          // log2(e) / sqrt(D)
   unsigned int epoch;        // launch id for bounded-wait abort propagation
 };
@@ -79,6 +88,41 @@ struct Params {
 __device__ __forceinline__ uint64_t kdesc(uint32_t saddr) { return umma_desc_sw128(saddr, 16, 1024); }
 __device__ __forceinline__ uint64_t vdesc(uint32_t saddr) { return umma_desc_sw128(saddr, HALF, 1024); }
 
+// One work item: a 128-row query tile of batch row b for query heads
+// h0 .. h0 + NH - 1 (all of KV group g). Items are numbered heaviest first
+// (highest query tile first); every role of a CTA derives the same items.
+struct Item {
+  int b, h0, g, q0, ds_last, kv_t0, n_kv;
+  int64_t rowbase;
+};
+
+__device__ __forceinline__ Item item_of(int item, const Params& p) {
+  Item it;
+  const int per_rank = p.B * p.n_hp;
+  const int qt = p.n_qt - 1 - item / per_rank;
+  const int rem = item % per_rank;
+  it.b = rem / p.n_hp;
+  it.h0 = (rem % p.n_hp) * p.NH;
+  it.g = it.h0 / p.G;
+  it.q0 = qt * BM;
+  const int q_last = min(it.q0 + BM - 1, p.S - 1);
+  it.rowbase = static_cast<int64_t>(it.b) * p.S;
+  const int ds_first = p.doc_start ? p.doc_start[it.rowbase + it.q0] : 0;
+  it.ds_last = p.doc_start ? p.doc_start[it.rowbase + q_last] : 0;
+  it.kv_t0 = ds_first / BN;
+  it.n_kv = qt - it.kv_t0 + 1;
+  return it;
+}
+
+// Persistent: one CTA per SM. Its first item is blockIdx.x; later ones are
+// claimed with an atomic counter (gridDim.x + counter), so items, numbered
+// heaviest first, are handed out first-come (longest-processing-time-first).
+// The producer publishes each claimed item id in a 4-entry shared-memory ring
+// before it arrives on the Q barrier; -1 ends every role's loop.
+// The K/V ring index and the per-tile barrier phases run on across items; the
+// next item's Q tiles are loaded as soon as the S MMAs of the current item have
+// finished reading Q, and the output tile is staged in the P buffer and stored
+// by warp 3, so one item's tail overlaps the next item's start.
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_bf16_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -88,25 +132,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t sbase = smem_addr(smem);
   const uint32_t bar0 = sbase + OFF_BAR;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * N_BARS);
+  volatile int* item_ring = reinterpret_cast<volatile int*>(smem + OFF_BAR + 8 * N_BARS + 8);
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtx wc{p.epoch};
-
-  // ---- work item: heaviest (highest) query tiles first
-  const int per_rank = p.B * p.n_hp;
-  const int qt = p.n_qt - 1 - static_cast<int>(blockIdx.x) / per_rank;
-  const int rem = static_cast<int>(blockIdx.x) % per_rank;
-  const int b = rem / p.n_hp, hp = rem % p.n_hp;
-  const int h0 = hp * p.NH;
-  const int g = h0 / p.G;
-  const int q0 = qt * BM;
-  const int q_last = min(q0 + BM - 1, p.S - 1);
-  const int64_t rowbase = static_cast<int64_t>(b) * p.S;
-  const int ds_first = p.doc_start ? p.doc_start[rowbase + q0] : 0;
-  const int ds_last = p.doc_start ? p.doc_start[rowbase + q_last] : 0;
-  const int kv_t0 = ds_first / BN;
-  const int n_kv = qt - kv_t0 + 1;
+  const int n_items = p.B * p.n_qt * p.n_hp;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
@@ -114,6 +145,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(bar(B_KV_EMPTY + s), 1);
     }
     mbar_init(bar(B_Q_FULL), 1);
+    mbar_init(bar(B_Q_FREE), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(B_Q_READY + s), 128);
       mbar_init(bar(B_S_READY + s), 1);
@@ -121,8 +153,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(bar(B_P_READY + s), 128);
       mbar_init(bar(B_PV_DONE + s), 1);
       mbar_init(bar(B_O_STAGED + s), 128);
+      mbar_init(bar(B_O_READ + s), 1);
     }
     mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_DRAIN_PV), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -139,14 +173,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(B_Q_FULL), static_cast<uint32_t>(p.NH) * TILE);
-      for (int s = 0; s < p.NH; ++s)
-        for (int hf = 0; hf < 2; ++hf)
-          tma_load_4d(sbase + OFF_Q + s * TILE + hf * HALF, &tm_q, bar(B_Q_FULL), hf * 64, h0 + s, q0, b);
-      uint32_t idx = 0;
-      auto load = [&](const CUtensorMap* tm, int kv_row) -> bool {
+      uint32_t idx = 0;  // running ring index
+      bool ok = true;
+      auto load = [&](const CUtensorMap* tm, int g, int kv_row, int b) -> bool {
         const uint32_t st = idx % NSTAGE, use = idx / NSTAGE;
         if (use > 0 && !mbar_wait(bar(B_KV_EMPTY + st), (use - 1) & 1, wc)) return false;
         mbar_arrive_expect_tx(bar(B_KV_FULL + st), TILE);
@@ -155,75 +186,145 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         ++idx;
         return true;
       };
-      bool ok = load(&tm_k, kv_t0 * BN);
-      for (int j = 1; ok && j < n_kv; ++j)
-        ok = load(&tm_k, (kv_t0 + j) * BN) && load(&tm_v, (kv_t0 + j - 1) * BN);
-      if (ok) load(&tm_v, (kv_t0 + n_kv - 1) * BN);
-      // Every issued load has landed before this CTA may exit (returns at once
-      // in the normal flow, where the MMA warp consumed them all).
-      mbar_wait(bar(B_Q_FULL), 0, wc);
+      int it = 0, item = blockIdx.x;
+      int next_item = (item < n_items) ? atomicAdd(p.sched, 1) + static_cast<int>(gridDim.x) : n_items;
+      bool ended = false;
+      for (;; ++it) {
+        if (it > 0 && !mbar_wait(bar(B_Q_FREE), (it - 1) & 1, wc)) {
+          ok = false;
+          break;
+        }
+        if (item >= n_items) {
+          item_ring[it & 3] = -1;
+          mbar_arrive(bar(B_Q_FULL));
+          ended = true;
+          break;
+        }
+        item_ring[it & 3] = item;
+        const Item I = item_of(item, p);
+        mbar_arrive_expect_tx(bar(B_Q_FULL), static_cast<uint32_t>(p.NH) * TILE);
+        for (int s = 0; s < p.NH; ++s)
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_4d(sbase + OFF_Q + s * TILE + hf * HALF, &tm_q, bar(B_Q_FULL), hf * 64, I.h0 + s, I.q0, I.b);
+        ok = load(&tm_k, I.g, I.kv_t0 * BN, I.b);
+        for (int j = 1; ok && j < I.n_kv; ++j)
+          ok = load(&tm_k, I.g, (I.kv_t0 + j) * BN, I.b) && load(&tm_v, I.g, (I.kv_t0 + j - 1) * BN, I.b);
+        if (ok) ok = load(&tm_v, I.g, (I.kv_t0 + I.n_kv - 1) * BN, I.b);
+        if (!ok) {
+          ++it;
+          break;
+        }
+        item = next_item;
+        next_item = (item < n_items) ? atomicAdd(p.sched, 1) + static_cast<int>(gridDim.x) : n_items;
+      }
+      // Every issued load has landed before this CTA may exit (these return at
+      // once in the normal flow, where every load was consumed).
+      if (!ended && it > 0) mbar_wait(bar(B_Q_FULL), (it - 1) & 1, wc);
       for (uint32_t st = 0; st < NSTAGE; ++st)
         if (idx > st) mbar_wait(bar(B_KV_FULL + st), ((idx - 1 - st) / NSTAGE) & 1, wc);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers
+    // Per item the load order is K0, K1, V0, K2, V1, ..., K(n-1), V(n-2), V(n-1):
+    // K_j sits at ring index base + (j == 0 ? 0 : 2j - 1) and V_j at
+    // base + (j < n-1 ? 2j + 2 : 2n - 1); base advances by 2n per item.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc_bf16_f32(128, 128, 0);
       constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 128, 1);
-      uint32_t idx = 0;
       bool ok = true;
-      for (int s = 0; s < p.NH; ++s) ok = ok && mbar_wait(bar(B_Q_READY + s), 0, wc);
-      auto next = [&](uint32_t& st) -> bool {
-        st = idx % NSTAGE;
-        const uint32_t use = idx / NSTAGE;
-        ++idx;
-        const bool r = mbar_wait(bar(B_KV_FULL + st), use & 1, wc);
-        tc_fence_after();
-        return r;
-      };
-      auto issue_s = [&](int j, uint32_t st) -> bool {
-        for (int s = 0; s < p.NH; ++s) {
-          if (j > 0 && !mbar_wait(bar(B_S_FREE + s), (j - 1) & 1, wc)) return false;
-          tc_fence_after();
-          const uint32_t qa = sbase + OFF_Q + s * TILE, kb = sbase + OFF_KV + st * TILE;
+      uint32_t ring = 0, tiles = 0;
+      for (int it = 0; ok; ++it) {
+        if (!mbar_wait(bar(B_Q_FULL), it & 1, wc)) break;
+        const int item = item_ring[it & 3];
+        if (item < 0) break;
+        const Item I = item_of(item, p);
+        if (warp == 1) {
+          for (int s = 0; s < p.NH; ++s) ok = ok && mbar_wait(bar(B_Q_READY + s), it & 1, wc);
+          for (int j = 0; ok && j < I.n_kv; ++j) {
+            const uint32_t idx = ring + ((j == 0) ? 0u : static_cast<uint32_t>(2 * j - 1));
+            const uint32_t st = idx % NSTAGE;
+            const uint32_t T = tiles + j;
+            if (!mbar_wait(bar(B_KV_FULL + st), (idx / NSTAGE) & 1, wc)) {
+              ok = false;
+              break;
+            }
+            const uint64_t db = kdesc(sbase + OFF_KV + st * TILE);
+            for (int s = 0; s < p.NH; ++s) {
+              if (T > 0 && !mbar_wait(bar(B_S_FREE + s), (T - 1) & 1, wc)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint64_t da = kdesc(sbase + OFF_Q + s * TILE);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * HALF + (kk & 3) * 32;
-            tc_mma_ss(tmem + s * 128, kdesc(qa + off), kdesc(kb + off), idesc_qk, kk > 0);
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t off = ((kk >> 2) * HALF + (kk & 3) * 32) >> 4;
+                tc_mma_ss(tmem + s * 128, da + off, db + off, idesc_qk, kk > 0);
+              }
+              tc_commit(bar(B_S_READY + s));
+            }
+            tc_commit(bar(B_KV_EMPTY + st));
           }
-          tc_commit(bar(B_S_READY + s));
-        }
-        tc_commit(bar(B_KV_EMPTY + st));
-        return true;
-      };
-      auto issue_pv = [&](int j, uint32_t st) -> bool {
-        for (int s = 0; s < p.NH; ++s) {
-          if (!mbar_wait(bar(B_P_READY + s), j & 1, wc)) return false;
-          tc_fence_after();
-          const uint32_t pa = sbase + OFF_P + s * TILE, vb = sbase + OFF_KV + st * TILE;
+          tc_commit(bar(B_Q_FREE));  // the Q tiles are free once these MMAs complete
+        } else {
+          for (int j = 0; ok && j < I.n_kv; ++j) {
+            const uint32_t idx =
+                ring + ((j < I.n_kv - 1) ? static_cast<uint32_t>(2 * j + 2) : static_cast<uint32_t>(2 * I.n_kv - 1));
+            const uint32_t st = idx % NSTAGE;
+            const uint32_t T = tiles + j;
+            if (!mbar_wait(bar(B_KV_FULL + st), (idx / NSTAGE) & 1, wc)) {
+              ok = false;
+              break;
+            }
+            const uint64_t db = vdesc(sbase + OFF_KV + st * TILE);
+            for (int s = 0; s < p.NH; ++s) {
+              if (!mbar_wait(bar(B_P_READY + s), T & 1, wc)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint64_t da = kdesc(sbase + OFF_P + s * TILE);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t aoff = (kk >> 2) * HALF + (kk & 3) * 32;
-            tc_mma_ss(tmem + 256 + s * 128, kdesc(pa + aoff), vdesc(vb + kk * 2048), idesc_pv,
-                      (j > 0 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t aoff = ((kk >> 2) * HALF + (kk & 3) * 32) >> 4;
+                tc_mma_ss(tmem + 256 + s * 128, da + aoff, db + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                          (j > 0 || kk > 0) ? 1u : 0u);
+              }
+              tc_commit(bar(B_PV_DONE + s));
+            }
+            tc_commit(bar(B_KV_EMPTY + st));
           }
-          tc_commit(bar(B_PV_DONE + s));
         }
-        tc_commit(bar(B_KV_EMPTY + st));
-        return true;
-      };
-      if (ok) {
-        uint32_t st;
-        ok = next(st) && issue_s(0, st);
-        for (int j = 1; ok && j < n_kv; ++j) {
-          ok = next(st) && issue_s(j, st);
-          ok = ok && next(st) && issue_pv(j - 1, st);
-        }
-        if (ok) ok = next(st) && issue_pv(n_kv - 1, st);
+        ring += 2u * static_cast<uint32_t>(I.n_kv);
+        tiles += static_cast<uint32_t>(I.n_kv);
       }
       // all issued MMAs complete before TMEM may be freed
-      tc_commit(bar(B_DRAIN));
-      mbar_wait(bar(B_DRAIN), 0, wc);
+      const int drain = (warp == 1) ? B_DRAIN : B_DRAIN_PV;
+      tc_commit(bar(drain));
+      mbar_wait(bar(drain), 0, wc);
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ output stores
+    if (lane == 0) {
+      bool ok = true;
+      for (int it = 0; ok; ++it) {
+        if (!mbar_wait(bar(B_O_STAGED + 0), it & 1, wc)) break;
+        const int item = item_ring[it & 3];
+        if (item < 0) break;
+        const Item I = item_of(item, p);
+        for (int s = 0; ok && s < p.NH; ++s) {
+          if (s > 0 && !mbar_wait(bar(B_O_STAGED + s), it & 1, wc)) {
+            ok = false;
+            break;
+          }
+          tma_store_4d(&tm_o, sbase + OFF_P + s * TILE, 0, I.h0 + s, I.q0, I.b);
+          tma_store_4d(&tm_o, sbase + OFF_P + s * TILE + HALF, 64, I.h0 + s, I.q0, I.b);
+          tma_store_commit();
+          tma_store_wait_read0();  // the P buffer may be rewritten from here on
+          mbar_arrive(bar(B_O_READ + s));
+        }
+      }
+      tma_store_wait0();
     }
   } else if (warp >= 4 && (warp - 4) / 4 < p.NH) {
     // ------------------------------------------------------------ softmax
@@ -233,124 +334,163 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + s * 128;
     const uint32_t tO = tmem + lane_off + 256 + s * 128;
-    const int qi = q0 + r;
-    const bool row_valid = qi < p.S;
-    const int qi_c = min(qi, p.S - 1);
-    const int ds_i = p.doc_start ? p.doc_start[rowbase + qi_c] : 0;
     uint8_t* qtile = smem + OFF_Q + s * TILE;
     uint8_t* ptile = smem + OFF_P + s * TILE;
-
-    bool ok = mbar_wait(bar(B_Q_FULL), 0, wc);
-    if (ok && row_valid) {
-      const float4* tab = p.rope_tab + static_cast<int64_t>(qi_c - ds_i) * 32;
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint4* ptr = reinterpret_cast<uint4*>(qtile + (c >> 3) * HALF + sw128_off(r, c & 7));
-        uint4 x = *ptr;
-        const float4 cs0 = __ldg(tab + 2 * c), cs1 = __ldg(tab + 2 * c + 1);
-        x.x = rope_rotate_pair(x.x, cs0.x, cs0.y);
-        x.y = rope_rotate_pair(x.y, cs0.z, cs0.w);
-        x.z = rope_rotate_pair(x.z, cs1.x, cs1.y);
-        x.w = rope_rotate_pair(x.w, cs1.z, cs1.w);
-        *ptr = x;
-      }
-    }
-    fence_proxy_async_smem();
-    mbar_arrive(bar(B_Q_READY + s));
-
     const float sl2 = p.scale_log2;
-    float m = -INFINITY;  // reference max, in log2 units of the scaled score
-    float l = 0.f;
-    for (int j = 0; ok && j < n_kv; ++j) {
-      const int kb = (kv_t0 + j) * BN;
-      if (!mbar_wait(bar(B_S_READY + s), j & 1, wc)) {
+    bool ok = true;
+    uint32_t tiles = 0;
+    for (int it = 0; ok; ++it) {
+      if (!mbar_wait(bar(B_Q_FULL), it & 1, wc)) {
         ok = false;
         break;
       }
-      tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-      tc_wait_ld();
-      tc_fence_before();
-      mbar_arrive(bar(B_S_FREE + s));
+      const int item = item_ring[it & 3];
+      if (item < 0) {
+        // tell the store warp the items are done, once it has read the last output
+        if (s == 0) {
+          if (it > 0) mbar_wait(bar(B_O_READ + 0), (it - 1) & 1, wc);
+          mbar_arrive(bar(B_O_STAGED + 0));
+        }
+        break;
+      }
+      const Item I = item_of(item, p);
+      const int qi = I.q0 + r;
+      const bool row_valid = qi < p.S;
+      const int qi_c = min(qi, p.S - 1);
+      const int ds_i = p.doc_start ? p.doc_start[I.rowbase + qi_c] : 0;
 
-      float sv[128];
+      if (row_valid) {
+        const float4* tab = p.rope_tab + static_cast<int64_t>(qi_c - ds_i) * 32;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c]);
-      if (kb + BN - 1 > q0 || kb < ds_last) {
-        const int lo = ds_i - kb, hi = qi_c - kb;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) sv[c] = (c < lo || c > hi) ? -INFINITY : sv[c];
+        for (int c = 0; c < 16; ++c) {
+          uint4* ptr = reinterpret_cast<uint4*>(qtile + (c >> 3) * HALF + sw128_off(r, c & 7));
+          uint4 x = *ptr;
+          const float4 cs0 = __ldg(tab + 2 * c), cs1 = __ldg(tab + 2 * c + 1);
+          x.x = rope_rotate_pair(x.x, cs0.x, cs0.y);
+          x.y = rope_rotate_pair(x.y, cs0.z, cs0.w);
+          x.z = rope_rotate_pair(x.z, cs1.x, cs1.y);
+          x.w = rope_rotate_pair(x.w, cs1.z, cs1.w);
+          *ptr = x;
+        }
       }
-      float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
-#pragma unroll
-      for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, sv[c]);
-        mx1 = fmaxf(mx1, sv[c + 1]);
-        mx2 = fmaxf(mx2, sv[c + 2]);
-        mx3 = fmaxf(mx3, sv[c + 3]);
-      }
-      const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-      const float m_new = fmaxf(m, mt);
-      const bool resc = m_new > m + kRescaleLog2;
-      float alpha = 1.f;
-      if (resc) {
-        alpha = ex2_approx(m - m_new);
-        m = m_new;
-      }
-      const float neg_m = (m == -INFINITY) ? 0.f : -m;
-      uint32_t pk[64];
-      float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = ex2_approx(fmaf(sv[c], sl2, neg_m));
-        const float p1 = ex2_approx(fmaf(sv[c + 1], sl2, neg_m));
-        rs0 += p0;
-        rs1 += p1;
-        pk[c >> 1] = pack_bf16x2(p0, p1);
-      }
-      l = l * alpha + (rs0 + rs1);
+      fence_proxy_async_smem();
+      mbar_arrive(bar(B_Q_READY + s));
 
-      if (j > 0) {
-        if (!mbar_wait(bar(B_PV_DONE + s), (j - 1) & 1, wc)) {
+      float m = -INFINITY;  // reference max, in log2 units of the scaled score
+      float l = 0.f;
+      for (int j = 0; j < I.n_kv; ++j) {
+        const int kb = (I.kv_t0 + j) * BN;
+        const uint32_t T = tiles + j;
+        if (!mbar_wait(bar(B_S_READY + s), T & 1, wc)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, resc)) {
-#pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t o[32];
-            tmem_ld32(tO + ch * 32, o);
-            tc_wait_ld();
-#pragma unroll
-            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-            tmem_st32(tO + ch * 32, o);
-          }
-          tc_wait_st();
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint4 w;
-        w.x = pk[4 * c];
-        w.y = pk[4 * c + 1];
-        w.z = pk[4 * c + 2];
-        w.w = pk[4 * c + 3];
-        *reinterpret_cast<uint4*>(ptile + (c >> 3) * HALF + sw128_off(r, c & 7)) = w;
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar(B_P_READY + s));
-    }
+        uint32_t sr[128];
+        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        tc_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(B_S_FREE + s));
 
-    // ---- epilogue: O / l -> bf16 -> Q tile buffer -> TMA store
-    if (ok) ok = mbar_wait(bar(B_PV_DONE + s), (n_kv - 1) & 1, wc);
-    tc_fence_after();
-    if (ok) {
+        float sv[128];
+#pragma unroll
+        for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c]);
+        if (kb + BN - 1 > I.q0 || kb < I.ds_last) {
+          const int lo = ds_i - kb, hi = qi_c - kb;
+#pragma unroll
+          for (int c = 0; c < 128; ++c) sv[c] = (c < lo || c > hi) ? -INFINITY : sv[c];
+        }
+        // four running maxima over columns a, a+4, ..., a+124 (a = 0..3)
+        float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+#pragma unroll
+        for (int c = 4; c <= 116; c += 8) {
+          mx0 = max3(mx0, sv[c], sv[c + 4]);
+          mx1 = max3(mx1, sv[c + 1], sv[c + 5]);
+          mx2 = max3(mx2, sv[c + 2], sv[c + 6]);
+          mx3 = max3(mx3, sv[c + 3], sv[c + 7]);
+        }
+        mx0 = fmaxf(mx0, sv[124]);
+        mx1 = fmaxf(mx1, sv[125]);
+        mx2 = fmaxf(mx2, sv[126]);
+        mx3 = fmaxf(mx3, sv[127]);
+        const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        const float m_new = fmaxf(m, mt);
+        const bool resc = m_new > m + kRescaleLog2;
+        float alpha = 1.f;
+        if (resc) {
+          alpha = ex2_approx(m - m_new);
+          m = m_new;
+        }
+        const float neg_m = (m == -INFINITY) ? 0.f : -m;
+        uint32_t pk[64];
+        // x = s * log2(e)/sqrt(D) - m and the running row sum in packed fp32 pairs
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), negmx2 = f2_pack(neg_m, neg_m);
+        uint64_t rsa = f2_pack(0.f, 0.f), rsb = rsa;
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sl2x2, negmx2), x0, x1);
+          // one pair in four goes through the FMA-pipe polynomial, the rest through MUFU
+          const bool poly = (c & 6) == 6;
+          const float p0 = poly ? ex2_poly(x0) : ex2_approx(x0);
+          const float p1 = poly ? ex2_poly(x1) : ex2_approx(x1);
+          if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));
+          else rsa = f2_add(rsa, f2_pack(p0, p1));
+          pk[c >> 1] = pack_bf16x2(p0, p1);
+        }
+        float rs0, rs1, rs2, rs3;
+        f2_unpack(rsa, rs0, rs1);
+        f2_unpack(rsb, rs2, rs3);
+        l = l * alpha + ((rs0 + rs2) + (rs1 + rs3));
+
+        if (j > 0) {
+          if (!mbar_wait(bar(B_PV_DONE + s), (T - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+              uint32_t o[32];
+              tmem_ld32(tO + ch * 32, o);
+              tc_wait_ld();
+#pragma unroll
+              for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+              tmem_st32(tO + ch * 32, o);
+            }
+            tc_wait_st();
+          }
+        } else if (it > 0 && !mbar_wait(bar(B_O_READ + s), (it - 1) & 1, wc)) {
+          // the previous item's output left the P buffer
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          uint4 w;
+          w.x = pk[4 * c];
+          w.y = pk[4 * c + 1];
+          w.z = pk[4 * c + 2];
+          w.w = pk[4 * c + 3];
+          *reinterpret_cast<uint4*>(ptile + (c >> 3) * HALF + sw128_off(r, c & 7)) = w;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(B_P_READY + s));
+      }
+      if (!ok) break;
+
+      // ---- epilogue: O / l -> bf16 -> P buffer; warp 3 stores it with TMA
+      const uint32_t T_last = tiles + I.n_kv - 1;
+      if (!mbar_wait(bar(B_PV_DONE + s), T_last & 1, wc)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
       const float inv_l = 1.f / l;
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
@@ -365,17 +505,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           w.z = pack_bf16x2(__uint_as_float(o[8 * c4 + 4]) * inv_l, __uint_as_float(o[8 * c4 + 5]) * inv_l);
           w.w = pack_bf16x2(__uint_as_float(o[8 * c4 + 6]) * inv_l, __uint_as_float(o[8 * c4 + 7]) * inv_l);
           const int d = ch * 32 + c4 * 8;
-          *reinterpret_cast<uint4*>(qtile + (d >> 6) * HALF + sw128_off(r, (d & 63) >> 3)) = w;
+          *reinterpret_cast<uint4*>(ptile + (d >> 6) * HALF + sw128_off(r, (d & 63) >> 3)) = w;
         }
       }
       fence_proxy_async_smem();
-    }
-    mbar_arrive(bar(B_O_STAGED + s));
-    if (r == 0 && ok && mbar_wait(bar(B_O_STAGED + s), 0, wc)) {
-      tma_store_4d(&tm_o, sbase + OFF_Q + s * TILE, 0, h0 + s, q0, b);
-      tma_store_4d(&tm_o, sbase + OFF_Q + s * TILE + HALF, 64, h0 + s, q0, b);
-      tma_store_commit();
-      tma_store_wait0();
+      tc_fence_before();
+      mbar_arrive(bar(B_O_STAGED + s));
+      tiles += static_cast<uint32_t>(I.n_kv);
     }
   }
 
