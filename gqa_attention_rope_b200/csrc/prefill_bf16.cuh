@@ -52,7 +52,7 @@ constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_KV = OFF_Q + 2 * TILE;
 constexpr uint32_t OFF_P = OFF_KV + NSTAGE * TILE;
 constexpr uint32_t OFF_BAR = OFF_P + 2 * TILE;
-constexpr uint32_t SMEM_USED = OFF_BAR + 256;
+constexpr uint32_t SMEM_USED = OFF_BAR + 512;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;
 constexpr int NTHREADS = 384;
 constexpr uint32_t TMEM_COLS = 512;
@@ -74,7 +74,8 @@ enum : int {
   B_DRAIN_PV,
   N_BARS
 };
-static_assert(N_BARS * 8 + 8 + 16 <= 256, "barrier area, TMEM address and item ring");
+constexpr int kItemRing = 8;
+static_assert(N_BARS * 8 + 8 + 8 * kItemRing <= 512, "barrier area, TMEM address and item ring");
 
 struct Params {
   int B, S, Hq, Hkv, G, NH, n_qt, n_hp;
@@ -117,8 +118,9 @@ __device__ __forceinline__ Item item_of(int item, const Params& p) {
 // Persistent: one CTA per SM. Its first item is blockIdx.x; later ones are
 // claimed with an atomic counter (gridDim.x + counter), so items, numbered
 // heaviest first, are handed out first-come (longest-processing-time-first).
-// The producer publishes each claimed item id in a 4-entry shared-memory ring
-// before it arrives on the Q barrier; -1 ends every role's loop.
+// The producer publishes each claimed item id in an 8-entry shared-memory ring
+// as soon as it is claimed (well before its Q tiles are loaded); -1 ends every
+// role's loop.
 // The K/V ring index and the per-tile barrier phases run on across items; the
 // next item's Q tiles are loaded as soon as the S MMAs of the current item have
 // finished reading Q, and the output tile is staged in the P buffer and stored
@@ -132,7 +134,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const uint32_t sbase = smem_addr(smem);
   const uint32_t bar0 = sbase + OFF_BAR;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * N_BARS);
-  volatile int* item_ring = reinterpret_cast<volatile int*>(smem + OFF_BAR + 8 * N_BARS + 8);
+  // item ring: slot k holds (item id, sequence number); the producer writes the
+  // item, then the sequence number; readers poll the sequence number.
+  volatile int* ring_item = reinterpret_cast<volatile int*>(smem + OFF_BAR + 8 * N_BARS + 8);
+  volatile int* ring_seq = ring_item + kItemRing;
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -157,6 +162,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     mbar_init(bar(B_DRAIN), 1);
     mbar_init(bar(B_DRAIN_PV), 1);
+    for (int k = 0; k < kItemRing; ++k) {  // no slot may look published before it is
+      ring_seq[k] = -1;
+      ring_item[k] = -1;
+    }
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -186,26 +195,46 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         ++idx;
         return true;
       };
+      // The RoPE table rows an item's Q rotation will read: positions
+      // q0 - ds(q0) .. +127 and, when a document starts inside the tile, 0 .. 127.
+      auto prefetch_rows = [&](int v) {
+        if (v < 0 || v >= n_items) return;
+        const Item J = item_of(v, p);
+        const int ds0 = p.doc_start ? p.doc_start[J.rowbase + J.q0] : 0;
+        const int p0 = J.q0 - ds0;
+        const int n0 = min(BM, p.S - p0);
+        if (n0 > 0) bulk_prefetch_l2(p.rope_tab + static_cast<int64_t>(p0) * 32, static_cast<uint32_t>(n0) * 512u);
+        if (J.ds_last > J.q0) bulk_prefetch_l2(p.rope_tab, static_cast<uint32_t>(min(BM, p.S)) * 512u);
+      };
+      auto publish = [&](int k, int v) {
+        ring_item[k % kItemRing] = v;
+        __threadfence_block();
+        ring_seq[k % kItemRing] = k;
+      };
       int it = 0, item = blockIdx.x;
       int next_item = (item < n_items) ? atomicAdd(p.sched, 1) + static_cast<int>(gridDim.x) : n_items;
       bool ended = false;
+      publish(0, item < n_items ? item : -1);
+      prefetch_rows(item);
       for (;; ++it) {
         if (it > 0 && !mbar_wait(bar(B_Q_FREE), (it - 1) & 1, wc)) {
           ok = false;
           break;
         }
         if (item >= n_items) {
-          item_ring[it & 3] = -1;
           mbar_arrive(bar(B_Q_FULL));
           ended = true;
           break;
         }
-        item_ring[it & 3] = item;
         const Item I = item_of(item, p);
         mbar_arrive_expect_tx(bar(B_Q_FULL), static_cast<uint32_t>(p.NH) * TILE);
         for (int s = 0; s < p.NH; ++s)
           for (int hf = 0; hf < 2; ++hf)
             tma_load_4d(sbase + OFF_Q + s * TILE + hf * HALF, &tm_q, bar(B_Q_FULL), hf * 64, I.h0 + s, I.q0, I.b);
+        item = next_item;
+        next_item = (item < n_items) ? atomicAdd(p.sched, 1) + static_cast<int>(gridDim.x) : n_items;
+        publish(it + 1, item < n_items ? item : -1);
+        prefetch_rows(item);
         ok = load(&tm_k, I.g, I.kv_t0 * BN, I.b);
         for (int j = 1; ok && j < I.n_kv; ++j)
           ok = load(&tm_k, I.g, (I.kv_t0 + j) * BN, I.b) && load(&tm_v, I.g, (I.kv_t0 + j - 1) * BN, I.b);
@@ -214,8 +243,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ++it;
           break;
         }
-        item = next_item;
-        next_item = (item < n_items) ? atomicAdd(p.sched, 1) + static_cast<int>(gridDim.x) : n_items;
       }
       // Every issued load has landed before this CTA may exit (these return at
       // once in the normal flow, where every load was consumed).
@@ -235,8 +262,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint32_t ring = 0, tiles = 0;
       for (int it = 0; ok; ++it) {
         if (!mbar_wait(bar(B_Q_FULL), it & 1, wc)) break;
-        const int item = item_ring[it & 3];
-        if (item < 0) break;
+        const int item = ring_item[it % kItemRing];
+        if (item < 0 || item >= n_items) break;
         const Item I = item_of(item, p);
         if (warp == 1) {
           for (int s = 0; s < p.NH; ++s) ok = ok && mbar_wait(bar(B_Q_READY + s), it & 1, wc);
@@ -309,8 +336,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       bool ok = true;
       for (int it = 0; ok; ++it) {
         if (!mbar_wait(bar(B_O_STAGED + 0), it & 1, wc)) break;
-        const int item = item_ring[it & 3];
-        if (item < 0) break;
+        const int item = ring_item[it % kItemRing];
+        if (item < 0 || item >= n_items) break;
         const Item I = item_of(item, p);
         for (int s = 0; ok && s < p.NH; ++s) {
           if (s > 0 && !mbar_wait(bar(B_O_STAGED + s), it & 1, wc)) {
@@ -339,43 +366,93 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
     uint32_t tiles = 0;
-    for (int it = 0; ok; ++it) {
+    Item I;
+    int qi_c = 0, ds_i = 0;
+    // Starts item `it`: reads its id from the ring, loads its row data, waits for
+    // its Q tile and rotates this thread's row in place. False at the end of the
+    // items (or on a timeout, which also clears ok).
+    auto begin_item = [&](int it) -> bool {
+      int item = -1;
+      {
+        const unsigned long long t0 = global_ns();
+        for (uint32_t k = 0;; ++k) {
+          if (ring_seq[it % kItemRing] == it) {
+            __threadfence_block();  // the item id was written before its sequence number
+            item = ring_item[it % kItemRing];
+            break;
+          }
+          if ((k & 63u) == 63u && (wc.aborted() || global_ns() - t0 > kWaitTimeoutNs)) {
+            if (!wc.aborted()) {
+              raise_error(LLAMA_ATTN_DEVERR_TIMEOUT);
+              atomicExch(&g_abort_epoch, wc.epoch);
+            }
+            ok = false;
+            return false;
+          }
+        }
+      }
+      if (item < 0) return false;
+      if (item >= n_items) {  // cannot happen unless the ring protocol is broken
+        raise_error(LLAMA_ATTN_DEVERR_TIMEOUT);
+        atomicExch(&g_abort_epoch, wc.epoch);
+        ok = false;
+        return false;
+      }
+      I = item_of(item, p);
+      const int qi = I.q0 + r;
+      qi_c = min(qi, p.S - 1);
+      ds_i = p.doc_start ? p.doc_start[I.rowbase + qi_c] : 0;
       if (!mbar_wait(bar(B_Q_FULL), it & 1, wc)) {
         ok = false;
-        break;
+        return false;
       }
-      const int item = item_ring[it & 3];
-      if (item < 0) {
-        // tell the store warp the items are done, once it has read the last output
-        if (s == 0) {
-          if (it > 0) mbar_wait(bar(B_O_READ + 0), (it - 1) & 1, wc);
-          mbar_arrive(bar(B_O_STAGED + 0));
-        }
-        break;
-      }
-      const Item I = item_of(item, p);
-      const int qi = I.q0 + r;
-      const bool row_valid = qi < p.S;
-      const int qi_c = min(qi, p.S - 1);
-      const int ds_i = p.doc_start ? p.doc_start[I.rowbase + qi_c] : 0;
-
-      if (row_valid) {
-        const float4* tab = p.rope_tab + static_cast<int64_t>(qi_c - ds_i) * 32;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          uint4* ptr = reinterpret_cast<uint4*>(qtile + (c >> 3) * HALF + sw128_off(r, c & 7));
-          uint4 x = *ptr;
-          const float4 cs0 = __ldg(tab + 2 * c), cs1 = __ldg(tab + 2 * c + 1);
-          x.x = rope_rotate_pair(x.x, cs0.x, cs0.y);
-          x.y = rope_rotate_pair(x.y, cs0.z, cs0.w);
-          x.z = rope_rotate_pair(x.z, cs1.x, cs1.y);
-          x.w = rope_rotate_pair(x.w, cs1.z, cs1.w);
-          *ptr = x;
+      // Rotate the warp's 32 Q rows two at a time: 16 lanes per row, 4 pairs
+      // per lane. A half-warp walks rows 2 apart; inside a document their
+      // positions are 2 apart too, so the (cos, sin) of the next row follow
+      // from the current ones by one rotation by 2*theta_k (angle addition,
+      // the table's row for position 2). The table is read only for the first
+      // row and where positions restart at a document start.
+      {
+        const int ch = lane & 15;
+        const float4* step = p.rope_tab + 2 * 32 + 2 * ch;
+        const float4 st0 = __ldg(step), st1 = __ldg(step + 1);
+        float4 c0 = make_float4(1.f, 0.f, 1.f, 0.f), c1 = c0;
+        int pos_prev = -4;
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int src = 2 * i + (lane >> 4);  // lane of the warp that owns the row
+          const int rr = wq * 32 + src;
+          const int pos = __shfl_sync(0xffffffffu, qi_c - ds_i, src);
+          if (pos == pos_prev + 2) {
+            c0 = make_float4(c0.x * st0.x - c0.y * st0.y, c0.y * st0.x + c0.x * st0.y,
+                             c0.z * st0.z - c0.w * st0.w, c0.w * st0.z + c0.z * st0.w);
+            c1 = make_float4(c1.x * st1.x - c1.y * st1.y, c1.y * st1.x + c1.x * st1.y,
+                             c1.z * st1.z - c1.w * st1.w, c1.w * st1.z + c1.z * st1.w);
+          } else {
+            const float4* tab = p.rope_tab + static_cast<int64_t>(pos) * 32 + 2 * ch;
+            c0 = __ldg(tab);
+            c1 = __ldg(tab + 1);
+          }
+          pos_prev = pos;
+          if (I.q0 + rr < p.S) {
+            uint4* ptr = reinterpret_cast<uint4*>(qtile + (ch >> 3) * HALF + sw128_off(rr, ch & 7));
+            uint4 x = *ptr;
+            x.x = rope_rotate_pair(x.x, c0.x, c0.y);
+            x.y = rope_rotate_pair(x.y, c0.z, c0.w);
+            x.z = rope_rotate_pair(x.z, c1.x, c1.y);
+            x.w = rope_rotate_pair(x.w, c1.z, c1.w);
+            *ptr = x;
+          }
         }
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(B_Q_READY + s));
+      return true;
+    };
 
+    bool more = begin_item(0);
+    const bool begin_ok_first = more;
+    for (int it = 0; ok && more; ++it) {
       float m = -INFINITY;  // reference max, in log2 units of the scaled score
       float l = 0.f;
       for (int j = 0; j < I.n_kv; ++j) {
@@ -484,14 +561,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       if (!ok) break;
 
+      // The next item's Q rotation overlaps the last PV of this one.
+      const Item cur = I;
+      const float l_cur = l;
+      more = begin_item(it + 1);
+      if (!ok) break;
+
       // ---- epilogue: O / l -> bf16 -> P buffer; warp 3 stores it with TMA
-      const uint32_t T_last = tiles + I.n_kv - 1;
+      const uint32_t T_last = tiles + cur.n_kv - 1;
       if (!mbar_wait(bar(B_PV_DONE + s), T_last & 1, wc)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      const float inv_l = 1.f / l_cur;
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         uint32_t o[32];
@@ -511,8 +594,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(B_O_STAGED + s));
-      tiles += static_cast<uint32_t>(I.n_kv);
+      tiles += static_cast<uint32_t>(cur.n_kv);
+      if (!more && ok && s == 0) {
+        // tell the store warp the items are done, once it has read the last output
+        mbar_wait(bar(B_O_READ + 0), it & 1, wc);
+        mbar_arrive(bar(B_O_STAGED + 0));
+      }
     }
+    if (ok && s == 0 && !begin_ok_first) mbar_arrive(bar(B_O_STAGED + 0));  // no items at all
   }
 
   tc_fence_before();
