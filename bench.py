@@ -63,13 +63,15 @@ class ClockSampler:
         self.max_mhz = None
 
     def _handle(self):
+        """NVML handle of this process's CUDA device, found by its PCI address
+        (CUDA and NVML may number devices differently)."""
         import pynvml
         pynvml.nvmlInit()
-        try:
-            bus = torch.cuda.get_device_properties(self.cuda_index).pci_bus_id
-            return pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode() if isinstance(bus, str) else bus)
-        except Exception:
-            return pynvml.nvmlDeviceGetHandleByIndex(self.cuda_index)
+        props = torch.cuda.get_device_properties(self.cuda_index)
+        dom, bus, dev = (getattr(props, n, None) for n in ("pci_domain_id", "pci_bus_id", "pci_device_id"))
+        if all(isinstance(x, int) for x in (dom, bus, dev)):
+            return pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08X}:{bus:02X}:{dev:02X}.0".encode())
+        return pynvml.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
     def start(self):
         import threading
