@@ -122,10 +122,12 @@ static int kv_head_of(int h, int Hq, int Hkv) { return h / (Hq / Hkv); }
  * Attention weights of one query row over the S keys of its batch row.
  * qrot: rotated query [D]; krot: rotated keys of the batch row [S, Hkv, D];
  * doc_start: row-local doc starts of the batch row [S]; i: the query's row index.
- * w receives S weights (masked keys get exactly 0).
+ * w receives S weights (masked keys get exactly 0). If lse is not NULL it
+ * receives log(sum over visible j of exp(s_ij)), the log of the softmax
+ * denominator of the scaled scores.
  */
 static void masked_softmax_row(const double *qrot, const double *krot, const int32_t *doc_start,
-                               int S, int Hkv, int g, int D, int i, double *w) {
+                               int S, int Hkv, int g, int D, int i, double *w, double *lse) {
   const double scale = 1.0 / sqrt((double)D);
   double m = -INFINITY;
   for (int j = 0; j < S; ++j) {
@@ -146,6 +148,7 @@ static void masked_softmax_row(const double *qrot, const double *krot, const int
     sum += w[j];
   }
   for (int j = 0; j < S; ++j) w[j] /= sum;
+  if (lse) *lse = m + log(sum);
 }
 
 /* Rotate every key of the batch at its token position: k [B*S, Hkv, D]. */
@@ -165,9 +168,10 @@ static double *rotate_keys(const double *k, const int32_t *pos_i, int64_t n_tok,
  * q_rows holds that token's query [n_rows, Hq, D]; rows == NULL means all B*S
  * tokens in order. out: [n_rows, Hq, D].
  */
-void oracle_prefill(const double *q_rows, const double *k, const double *v,
-                    const int32_t *doc_start, const int32_t *pos, int B, int S, int Hq, int Hkv,
-                    int D, double base, const int64_t *rows, int64_t n_rows, double *out) {
+static void prefill_impl(const double *q_rows, const double *k, const double *v,
+                         const int32_t *doc_start, const int32_t *pos, int B, int S, int Hq, int Hkv,
+                         int D, double base, const int64_t *rows, int64_t n_rows, double *out,
+                         double *lse_out) {
   const int64_t n_tok = (int64_t)B * S;
   double *krot = rotate_keys(k, pos, n_tok, Hkv, D, base);
   double *freqs = (double *)malloc(sizeof(double) * (size_t)(D / 2));
@@ -186,7 +190,8 @@ void oracle_prefill(const double *q_rows, const double *k, const double *v,
       const int g = kv_head_of(h, Hq, Hkv);
       rope_rotate_one(q_rows + (r * Hq + h) * D, qrot, D, (double)pos[t], freqs);
       const double *krow = krot + (int64_t)b * S * Hkv * D;
-      masked_softmax_row(qrot, krow, doc_start + (int64_t)b * S, S, Hkv, g, D, i, w);
+      masked_softmax_row(qrot, krow, doc_start + (int64_t)b * S, S, Hkv, g, D, i, w,
+                         lse_out ? lse_out + r * Hq + h : NULL);
       double *o = out + (r * Hq + h) * D;
       for (int d = 0; d < D; ++d) o[d] = 0.0;
       const double *vrow = v + (int64_t)b * S * Hkv * D;
@@ -201,6 +206,24 @@ void oracle_prefill(const double *q_rows, const double *k, const double *v,
   }
   free(freqs);
   free(krot);
+}
+
+void oracle_prefill(const double *q_rows, const double *k, const double *v,
+                    const int32_t *doc_start, const int32_t *pos, int B, int S, int Hq, int Hkv,
+                    int D, double base, const int64_t *rows, int64_t n_rows, double *out) {
+  prefill_impl(q_rows, k, v, doc_start, pos, B, S, Hq, Hkv, D, base, rows, n_rows, out, NULL);
+}
+
+/*
+ * Prefill that also returns, per query row and head, the log-sum-exp of its
+ * visible scaled scores: lse [n_rows, Hq] (natural logarithm). This is the
+ * quantity that lets partial attentions over disjoint key sets be merged.
+ */
+void oracle_prefill_lse(const double *q_rows, const double *k, const double *v,
+                        const int32_t *doc_start, const int32_t *pos, int B, int S, int Hq, int Hkv,
+                        int D, double base, const int64_t *rows, int64_t n_rows, double *out,
+                        double *lse) {
+  prefill_impl(q_rows, k, v, doc_start, pos, B, S, Hq, Hkv, D, base, rows, n_rows, out, lse);
 }
 
 /*
@@ -219,7 +242,7 @@ void oracle_prefill_weights(const double *q, const double *k, const int32_t *doc
   const int64_t t = (int64_t)b * S + i;
   rope_rotate_one(q + (t * Hq + h) * D, qrot, D, (double)pos[t], freqs);
   masked_softmax_row(qrot, krot + (int64_t)b * S * Hkv * D, doc_start + (int64_t)b * S, S, Hkv,
-                     kv_head_of(h, Hq, Hkv), D, i, w);
+                     kv_head_of(h, Hq, Hkv), D, i, w, NULL);
   free(qrot);
   free(freqs);
   free(krot);

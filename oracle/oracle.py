@@ -46,6 +46,8 @@ def load_library(path: str):
     lib.oracle_prefill.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, f64, P, i64, P]
     lib.oracle_prefill_weights.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, f64, i32, i32, i32, P]
     lib.oracle_decode.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, f64, P]
+    if hasattr(lib, "oracle_prefill_lse"):
+        lib.oracle_prefill_lse.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, f64, P, i64, P, P]
     return lib
 
 
@@ -151,6 +153,31 @@ def prefill(q, k, v, doc_offsets=None, rope_theta: float = 500000.0, rows=None, 
     lib.oracle_prefill(_p(qf), _p(kf), _p(vf), _p(ds), _p(pos), B, S, Hq, Hkv, D, float(rope_theta),
                        None if rows_arr is None else _p(rows_arr), n_rows, _p(out))
     return out.reshape(B, S, Hq, D) if rows is None else out
+
+
+def prefill_lse(q, k, v, doc_offsets=None, rope_theta: float = 500000.0, rows=None, lib=None):
+    """(out, lse): attention output and the per-row, per-head log-sum-exp of
+    the visible scaled scores (natural log). Shapes as in prefill; lse is
+    [B, S, Hq] or [len(rows), Hq]."""
+    lib = lib or _get()
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    ds, pos = doc_layout(doc_offsets, B, S, lib)
+    kf, vf = _f64(k), _f64(v)
+    if rows is None:
+        qf = _f64(q).reshape(B * S, Hq, D)
+        n_rows, rows_arr = B * S, None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        n_rows = rows_arr.shape[0]
+        qf = _f64(_take_rows(q.reshape(B * S, Hq, D), rows_arr))
+    out = np.empty((n_rows, Hq, D), np.float64)
+    lse = np.empty((n_rows, Hq), np.float64)
+    lib.oracle_prefill_lse(_p(qf), _p(kf), _p(vf), _p(ds), _p(pos), B, S, Hq, Hkv, D, float(rope_theta),
+                           None if rows_arr is None else _p(rows_arr), n_rows, _p(out), _p(lse))
+    if rows is None:
+        return out.reshape(B, S, Hq, D), lse.reshape(B, S, Hq)
+    return out, lse
 
 
 def prefill_weights(q, k, b: int, h: int, i: int, doc_offsets=None, rope_theta: float = 500000.0,

@@ -294,6 +294,32 @@ def check_doc_layout(lib):
         raise AssertionError(f"accepted malformed offsets {b}")
 
 
+def check_lse(lib):
+    """The log-sum-exp the oracle reports equals torch.logsumexp of the
+    independently formed masked scores, and out = sum exp(s - lse) v."""
+    if not hasattr(lib, "oracle_prefill_lse"):
+        return
+    gen = torch.Generator().manual_seed(18)
+    B, S, Hq, Hkv, D, base = 2, 14, 4, 2, 8, 500000.0
+    lens = [[5, 9], [14]]
+    q, k, v = _rand(gen, B, S, Hq, D), _rand(gen, B, S, Hkv, D), _rand(gen, B, S, Hkv, D)
+    out, lse = O.prefill_lse(q, k, v, offsets_of(lens, S), base, lib=lib)
+    doc, pos = torch_doc_ids_positions(lens, S)
+    qr = torch_rope_complex(q, pos, base)
+    kr = torch_rope_complex(k, pos, base).repeat_interleave(Hq // Hkv, dim=2)
+    vr = v.repeat_interleave(Hq // Hkv, dim=2)
+    scores = torch.einsum("bihd,bjhd->bhij", qr, kr) / math.sqrt(D)
+    i = torch.arange(S)
+    mask = (doc[:, :, None] == doc[:, None, :]) & (i[None, None, :] <= i[None, :, None])
+    scores = scores.masked_fill(~mask[:, None], float("-inf"))
+    ref = torch.logsumexp(scores, dim=-1).permute(0, 2, 1)  # [B, S, Hq]
+    assert np.allclose(lse, ref.numpy(), rtol=1e-12, atol=1e-12)
+    rebuilt = torch.einsum("bhij,bjhd->bihd", torch.exp(scores - ref.permute(0, 2, 1)[..., None]), vr)
+    assert np.allclose(out, rebuilt.numpy(), rtol=1e-11, atol=1e-11)
+    # the plain entry point gives the same output
+    assert np.array_equal(out, O.prefill(q, k, v, offsets_of(lens, S), base, lib=lib))
+
+
 ALL_CHECKS = [
     check_rope_freqs_closed_form,
     check_rope_identities,
@@ -305,4 +331,5 @@ ALL_CHECKS = [
     check_softmax_invariants,
     check_decode_consistent_with_prefill,
     check_doc_layout,
+    check_lse,
 ]

@@ -35,6 +35,7 @@ MUTANTS = {
     "decode_scale": ("s[n] = dot * scale;", "s[n] = dot;"),
     "doc_position_not_restarted_inside_row": ("pos[t] = (int32_t)(t - start);",
                                               "pos[t] = (int32_t)(t - start + (t - start) / 2);"),
+    "lse_drops_max": ("if (lse) *lse = m + log(sum);", "if (lse) *lse = log(sum);"),
 }
 
 
