@@ -27,6 +27,7 @@ EXPORTED = (
     "llama_attn_profile_begin",
     "llama_attn_profile_end",
     "llama_attn_decode_noalloc",
+    "llama_attn_prefill_ex",
 )
 
 DEVERR_TIMEOUT = 0x1
@@ -71,6 +72,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.llama_attn_profile_end.restype = I
     lib.llama_attn_decode_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, F, P]
     lib.llama_attn_decode_noalloc.restype = I
+    lib.llama_attn_prefill_ex.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P, P, I, P]
+    lib.llama_attn_prefill_ex.restype = I
     return lib
 
 
@@ -149,6 +152,38 @@ def llama_attn_prefill(q, k, v, out=None, doc_offsets=None, rope_theta: float = 
                                   float(rope_theta), _stream(stream))
     _check("llama_attn_prefill", st)
     return out
+
+
+def llama_attn_prefill_ex(q, k, v, out=None, lse=None, doc_offsets=None, rope_theta: float = 500000.0,
+                          kcache=None, vcache=None, stream=None):
+    """bf16 prefill that can also return the per-row log-sum-exp (``lse``,
+    float32 [B, S, Hq]) and append rotated K and V to a decode-layout cache
+    (``kcache``/``vcache`` [B, Hkv, Lmax, D]). Returns (out, lse)."""
+    import torch
+    _require(q.dim() == 4 and k.dim() == 4 and v.dim() == 4, "q, k, v must be [B, S, H, D]")
+    for t in (q, k, v):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "bf16 contiguous CUDA tensors expected")
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _require(k.shape == (B, S, Hkv, D) and v.shape == k.shape, "k and v must be [B, S, Hkv, D]")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is not None:
+        _require(lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.shape == (B, S, Hq),
+                 "lse: float32 [B, S, Hq]")
+    Lmax = 0
+    if kcache is not None or vcache is not None:
+        _require(kcache is not None and vcache is not None and kcache.shape == vcache.shape, "kcache and vcache")
+        for t in (kcache, vcache):
+            _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "bf16 contiguous caches")
+        _require(kcache.shape[0] == B and kcache.shape[1] == Hkv and kcache.shape[3] == D, "cache shape")
+        Lmax = kcache.shape[2]
+    if doc_offsets is not None:
+        _require(doc_offsets.is_cuda and doc_offsets.dtype == torch.int32, "doc_offsets: int32 CUDA tensor")
+    st = lib().llama_attn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(doc_offsets), B, S, Hq,
+                                     Hkv, D, float(rope_theta), _ptr(kcache), _ptr(vcache), Lmax, _stream(stream))
+    _check("llama_attn_prefill_ex", st)
+    return out, lse
 
 
 def llama_attn_prefill_f32(q, k, v, out=None, doc_offsets=None, rope_theta: float = 500000.0, stream=None):

@@ -287,13 +287,23 @@ int llama_attn_get_device_error(cudaStream_t stream) {
   return err;
 }
 
-int llama_attn_prefill(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
-                       llama_attn_bf16* out, const int32_t* doc_offsets, int B, int S, int Hq, int Hkv, int D,
-                       float rope_theta, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// bf16 prefill shared by llama_attn_prefill and llama_attn_prefill_ex: lse,
+// kcache and vcache may be null (no log-sum-exp output, no cache append).
+int prefill_bf16_impl(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
+                      llama_attn_bf16* out, float* lse, const int32_t* doc_offsets, int B, int S, int Hq, int Hkv,
+                      int D, float rope_theta, llama_attn_bf16* kcache, llama_attn_bf16* vcache, int Lmax,
+                      cudaStream_t stream) {
   int st = check_prefill_common(q, k, v, out, B, S, Hq, Hkv, rope_theta);
   if (st) return st;
   if (D != 128) return LLAMA_ATTN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if ((kcache == nullptr) != (vcache == nullptr)) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (kcache && (Lmax < S || !aligned16(kcache) || !aligned16(vcache))) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LLAMA_ATTN_ERR_INVALID_ARG;
   if (static_cast<int64_t>(S) * Hq * 256 >= (int64_t(1) << 40)) return LLAMA_ATTN_ERR_UNSUPPORTED;
   int dev;
   if ((st = current_device(&dev))) return st;
@@ -319,6 +329,13 @@ int llama_attn_prefill(const llama_attn_bf16* q, const llama_attn_bf16* k, const
       reinterpret_cast<const uint4*>(k), reinterpret_cast<uint4*>(dc.krot), reinterpret_cast<const float4*>(tab),
       doc_start, S, Hkv, nvec);
   LA_CUDA(cudaGetLastError());
+  if (kcache) {
+    prof_count(1);
+    la::kv_cache_append_kernel<<<grid_for(nvec, 256), 256, 0, stream>>>(
+        reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), reinterpret_cast<const float4*>(tab),
+        doc_start, reinterpret_cast<uint4*>(kcache), reinterpret_cast<uint4*>(vcache), S, Hkv, Lmax, nvec);
+    LA_CUDA(cudaGetLastError());
+  }
 
   CUtensorMap tq, tk, tv, to;
   if ((st = tmap_bshd(&tq, q, B, S, Hq))) return st;
@@ -342,6 +359,7 @@ int llama_attn_prefill(const llama_attn_bf16* q, const llama_attn_bf16* k, const
   if (dc.sched == nullptr) LA_CUDA(cudaMalloc(&dc.sched, 256));
   LA_CUDA(cudaMemsetAsync(dc.sched, 0, sizeof(int), stream));
   p.sched = dc.sched;
+  p.lse = lse;
   const int64_t items = static_cast<int64_t>(B) * p.n_qt * p.n_hp;
   if (items > INT32_MAX) return LLAMA_ATTN_ERR_UNSUPPORTED;
   if (!dc.prefill_attr_set) {
@@ -358,6 +376,25 @@ int llama_attn_prefill(const llama_attn_bf16* q, const llama_attn_bf16* k, const
   const cudaError_t e = cudaGetLastError();
   prof_after(pair, stream);
   return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int llama_attn_prefill(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
+                       llama_attn_bf16* out, const int32_t* doc_offsets, int B, int S, int Hq, int Hkv, int D,
+                       float rope_theta, cudaStream_t stream) {
+  return prefill_bf16_impl(q, k, v, out, nullptr, doc_offsets, B, S, Hq, Hkv, D, rope_theta, nullptr, nullptr, 0,
+                           stream);
+}
+
+int llama_attn_prefill_ex(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
+                          llama_attn_bf16* out, float* lse, const int32_t* doc_offsets, int B, int S, int Hq,
+                          int Hkv, int D, float rope_theta, llama_attn_bf16* kcache, llama_attn_bf16* vcache,
+                          int Lmax, cudaStream_t stream) {
+  return prefill_bf16_impl(q, k, v, out, lse, doc_offsets, B, S, Hq, Hkv, D, rope_theta, kcache, vcache, Lmax,
+                           stream);
 }
 
 int llama_attn_prefill_f32(const float* q, const float* k, const float* v, float* out, const int32_t* doc_offsets,

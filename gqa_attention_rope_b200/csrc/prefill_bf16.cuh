@@ -82,6 +82,7 @@ struct Params {
   const int32_t* doc_start;  // [B*S] row-local document start, or null (one document per row)
   const float4* rope_tab;    // (cos, sin) pairs, 64 per position, as float4 = 2 pairs
   int* sched;                // work-item counter, zero at launch
+  float* lse;                // optional [B*S, Hq] log-sum-exp of each row's visible scaled scores
   float scale_log2;          // log2(e) / sqrt(D)
   unsigned int epoch;        // launch id for bounded-wait abort propagation
 };
@@ -594,6 +595,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(B_O_STAGED + s));
+      if (p.lse != nullptr && cur.q0 + r < p.S)  // natural log: ln 2 * (m + log2 l)
+        p.lse[(cur.rowbase + cur.q0 + r) * p.Hq + cur.h0 + s] = 0.69314718055994531f * (m + log2f(l_cur));
       tiles += static_cast<uint32_t>(cur.n_kv);
       if (!more && ok && s == 0) {
         // tell the store warp the items are done, once it has read the last output

@@ -104,4 +104,35 @@ __global__ void rope_rotate_rows_bf16_kernel(const uint4* __restrict__ x, uint4*
   }
 }
 
+// Appends a prefill batch to a decode-layout KV cache: token i of batch row b
+// and KV head h goes to cache row i of (b, h), the key rotated at the token's
+// document position (position i when the row is one document), the value
+// copied. k, v: [B, S, H, 128]; kcache, vcache: [B, H, Lmax, 128], Lmax >= S.
+// One thread per 16-byte vector (4 pairs).
+__global__ void kv_cache_append_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                       const float4* __restrict__ tab, const int32_t* __restrict__ doc_start,
+                                       uint4* __restrict__ kcache, uint4* __restrict__ vcache, int S, int H,
+                                       int Lmax, int64_t n_vec) {
+  constexpr int kVecPerRow = 16;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < n_vec;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = idx / (static_cast<int64_t>(H) * kVecPerRow);
+    const int rem = static_cast<int>(idx % (static_cast<int64_t>(H) * kVecPerRow));
+    const int h = rem / kVecPerRow, c = rem % kVecPerRow;
+    const int64_t b = t / S;
+    const int i = static_cast<int>(t % S);
+    const int pos = i - (doc_start ? doc_start[t] : 0);
+    const float4* tp = tab + static_cast<int64_t>(pos) * 32 + c * 2;
+    const float4 cs0 = __ldg(tp), cs1 = __ldg(tp + 1);
+    uint4 kv = k[idx];
+    kv.x = rope_rotate_pair(kv.x, cs0.x, cs0.y);
+    kv.y = rope_rotate_pair(kv.y, cs0.z, cs0.w);
+    kv.z = rope_rotate_pair(kv.z, cs1.x, cs1.y);
+    kv.w = rope_rotate_pair(kv.w, cs1.z, cs1.w);
+    const int64_t dst = ((b * H + h) * Lmax + i) * kVecPerRow + c;
+    kcache[dst] = kv;
+    vcache[dst] = v[idx];
+  }
+}
+
 }  // namespace la

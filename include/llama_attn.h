@@ -84,6 +84,31 @@ int llama_attn_prefill(const llama_attn_bf16 *q, const llama_attn_bf16 *k,
                        float rope_theta, cudaStream_t stream);
 
 /*
+ * llama_attn_prefill plus the two outputs that link prefill to decode:
+ *
+ *   lse    [B, S, Hq] float32, or NULL: per query row and head, the natural
+ *          log of the softmax denominator over the row's visible keys,
+ *          log(sum_j exp(q_i . k_j / sqrt(D))) with rotated q and k. With it,
+ *          attention over disjoint key sets can be merged exactly.
+ *   kcache, vcache  [B, Hkv, Lmax, D] bf16, or both NULL: the batch is
+ *          appended to a decode-layout KV cache, token i of batch row b and KV
+ *          head h going to cache row i of (b, h): the key rotated at the
+ *          token's document position (position i when doc_offsets is NULL,
+ *          which is the form a following llama_attn_decode continues from at
+ *          cache_lens[b] = S), the value copied. Rows S .. Lmax-1 are not
+ *          touched. Lmax >= S.
+ *
+ * The attention output equals llama_attn_prefill's. Errors as for
+ * llama_attn_prefill; a cache pointer without the other, Lmax < S or a cache
+ * not 16-byte aligned returns LLAMA_ATTN_ERR_INVALID_ARG.
+ */
+int llama_attn_prefill_ex(const llama_attn_bf16 *q, const llama_attn_bf16 *k,
+                          const llama_attn_bf16 *v, llama_attn_bf16 *out, float *lse,
+                          const int32_t *doc_offsets, int B, int S, int Hq, int Hkv, int D,
+                          float rope_theta, llama_attn_bf16 *kcache, llama_attn_bf16 *vcache,
+                          int Lmax, cudaStream_t stream);
+
+/*
  * Prefill in true fp32 arithmetic on CUDA cores (FFMA, accurate expf), same
  * semantics and layouts as llama_attn_prefill with float tensors.
  * D even, 2 <= D <= 128.
