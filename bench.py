@@ -346,6 +346,38 @@ def run_decode(args, la, dev, world, rank, hbm_peak, peak_kind):
     def step():
         la.llama_attn_decode(q, kc, vc, lens, out=out, workspace=ws, rope_theta=w.rope_theta)
 
+    if args.decode_page_size:
+        # the same cache rows scattered over a page pool by a fixed permutation
+        import ctypes
+        P = args.decode_page_size
+        max_blocks = (w.Lmax + P - 1) // P
+        need = [(int(n) + P - 1) // P for n in inp["cache_lens"]]
+        n_pages = sum(need)
+        perm = torch.randperm(n_pages, generator=torch.Generator().manual_seed(1234)).tolist()
+        kp = torch.empty((n_pages, w.Hkv, P, w.D), dtype=torch.bfloat16, device=dev)
+        vp = torch.empty_like(kp)
+        table = torch.full((w.B, max_blocks), -1, dtype=torch.int32)
+        it = iter(perm)
+        for b in range(w.B):
+            for j in range(need[b]):
+                pg = next(it)
+                table[b, j] = pg
+                lo, hi = j * P, min((j + 1) * P, w.Lmax)
+                kp[pg, :, :hi - lo] = kc[b, :, lo:hi]
+                vp[pg, :, :hi - lo] = vc[b, :, lo:hi]
+        table = table.to(dev)
+        del kc, vc
+        torch.cuda.empty_cache()
+        lib = la.lib()
+        sptr = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+
+        def step():  # noqa: F811
+            st = lib.llama_attn_decode_paged(ptr(q), ptr(kp), ptr(vp), ptr(table), ptr(lens), ptr(out), w.B, w.Hq,
+                                             w.Hkv, w.D, P, max_blocks, n_pages, ctypes.c_float(w.rope_theta),
+                                             ptr(ws), ws.numel(), sptr)
+            assert st == 0
+
     for _ in range(5):
         step()
     torch.cuda.synchronize()
@@ -365,7 +397,8 @@ def run_decode(args, la, dev, world, rank, hbm_peak, peak_kind):
     kernel_ms = main_ms / max(main_n, 1)
     achieved = kv_bytes / (kernel_ms / 1e3) / 1e9
     return {
-        "workload": w.name, "value": all_bytes / (total_ms / 1e3) / 1e9, "unit": "GB/s", "steps": steps,
+        "workload": w.name + (f"_paged{args.decode_page_size}" if args.decode_page_size else ""),
+        "value": all_bytes / (total_ms / 1e3) / 1e9, "unit": "GB/s", "steps": steps,
         "ms_per_step": total_ms / steps, "bytes_per_step_per_gpu": kv_bytes + io_bytes, "cache_tokens": tokens,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_kind": f"{peak_kind} HBM copy",
@@ -404,6 +437,8 @@ def main():
     ap.add_argument("--decode-seqs", type=int, default=W.DECODE_70B.B,
                     help="sequences in the decode batch (64 = the 70B-shaped workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode-page-size", type=int, default=0,
+                    help="time the decode through the paged-cache entry point with this page size")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args()
     w = W.WORKLOADS[args.workload]

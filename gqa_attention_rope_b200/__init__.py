@@ -28,11 +28,13 @@ EXPORTED = (
     "llama_attn_profile_end",
     "llama_attn_decode_noalloc",
     "llama_attn_prefill_ex",
+    "llama_attn_decode_paged",
 )
 
 DEVERR_TIMEOUT = 0x1
 DEVERR_DOC_OFFSETS = 0x2
 DEVERR_CACHE_LEN = 0x4
+DEVERR_BLOCK_TABLE = 0x8
 
 _lock = threading.Lock()
 _lib = None
@@ -74,6 +76,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.llama_attn_decode_noalloc.restype = I
     lib.llama_attn_prefill_ex.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, P, P, I, P]
     lib.llama_attn_prefill_ex.restype = I
+    lib.llama_attn_decode_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, P, Z, P]
+    lib.llama_attn_decode_paged.restype = I
     return lib
 
 

@@ -50,6 +50,11 @@ struct Params {
   float* part_lse;           // [B, Hq, nchunk]
   unsigned int epoch;        // launch id for bounded-wait abort propagation
   double rope_theta;         // used only when the kernel forms its own (cos, sin) row
+  // paged cache (kPaged): logical row n of sequence b lives in page
+  // block_table[b * max_blocks + n / page_size] at row n % page_size; the page
+  // pool is [n_pages, Hkv, page_size, 128], page_size a multiple of ROWS.
+  const int32_t* block_table;
+  int page_size, max_blocks, n_pages;
 };
 
 __device__ __forceinline__ int valid_len(int len, int Lmax) { return (len < 0 || len > Lmax) ? 0 : len; }
@@ -58,7 +63,7 @@ __device__ __forceinline__ int valid_len(int len, int Lmax) { return (len < 0 ||
 // p.rope_tab. kSelfTable = true: the CTA forms that one row itself (float64
 // angle, same formula as rope_table_kernel) in shared memory, so no table needs
 // to be allocated.
-template <bool kSelfTable>
+template <bool kSelfTable, bool kPaged = false>
 __global__ void __launch_bounds__(NTHREADS, 2)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const Params p) {
@@ -75,7 +80,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   if (n0 >= len) return;
   const int n1 = min(len, n0 + CHUNK);
   const int nst = (n1 - n0 + ROWS - 1) / ROWS;
-  const int row0 = (b * p.Hkv + gk) * p.Lmax + n0;
+  const int row0 = kPaged ? 0 : (b * p.Hkv + gk) * p.Lmax + n0;  // contiguous layout only
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WaitCtx wc{p.epoch};
 
@@ -107,7 +112,18 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         if (use > 0 && !mbar_wait(empty(st), (use - 1) & 1, wc)) break;
         mbar_arrive_expect_tx(full(st), STAGE);
         const uint32_t dst = sbase + st * STAGE;
-        const int r = row0 + i * ROWS;
+        int r = row0 + i * ROWS;
+        if constexpr (kPaged) {
+          // a stage of ROWS rows lies inside one page (page_size is a multiple of ROWS)
+          const int n = n0 + i * ROWS;
+          const int page = p.block_table[static_cast<int64_t>(b) * p.max_blocks + n / p.page_size];
+          if (page < 0 || page >= p.n_pages) {
+            raise_error(LLAMA_ATTN_DEVERR_BLOCK_TABLE);
+            r = p.n_pages * p.Hkv * p.page_size;  // past the pool: TMA reads zeros
+          } else {
+            r = (page * p.Hkv + gk) * p.page_size + n % p.page_size;
+          }
+        }
         tma_load_2d(dst, &tm_k, full(st), 0, r);
         tma_load_2d(dst + KHALF, &tm_k, full(st), 64, r);
         tma_load_2d(dst + 2 * KHALF, &tm_v, full(st), 0, r);

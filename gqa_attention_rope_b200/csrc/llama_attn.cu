@@ -37,6 +37,7 @@ struct DeviceCache {
   int* sched = nullptr;  // work-item counter of the persistent prefill kernel
   bool prefill_attr_set = false;
   bool decode_attr_set = false;
+  bool decode_paged_attr_set = false;
 };
 
 std::mutex g_mutex;
@@ -549,6 +550,72 @@ int llama_attn_decode_noalloc(const llama_attn_bf16* q, const llama_attn_bf16* k
   const dim3 grid(p.nchunk, Hkv, B);
   la::dec::decode_split_kernel<true><<<grid, la::dec::NTHREADS, la::dec::SMEM_ALLOC_SELF_TABLE, stream>>>(tk, tv, p);
   LA_CUDA(cudaGetLastError());
+  la::dec::decode_combine_kernel<<<B * Hq, 128, 0, stream>>>(p.part_o, p.part_lse, cache_lens, out, Hq, Lmax,
+                                                            p.nchunk);
+  return cuda_status(cudaGetLastError());
+}
+
+int llama_attn_decode_paged(const llama_attn_bf16* q, const llama_attn_bf16* kpages, const llama_attn_bf16* vpages,
+                            const int32_t* block_table, const int32_t* cache_lens, llama_attn_bf16* out, int B,
+                            int Hq, int Hkv, int D, int page_size, int max_blocks, int n_pages, float rope_theta,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!q || !kpages || !vpages || !block_table || !cache_lens || !out) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (page_size <= 0 || max_blocks <= 0 || n_pages <= 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.f) || !std::isfinite(rope_theta)) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (D != 128 || Hq / Hkv > 16 || page_size % la::dec::ROWS != 0) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  if (B > 65535 || Hkv > 65535 || B * Hq > INT32_MAX / 2) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  const int64_t Lmax64 = static_cast<int64_t>(max_blocks) * page_size;
+  if (Lmax64 >= INT32_MAX || static_cast<int64_t>(n_pages) * Hkv * page_size >= INT32_MAX - page_size)
+    return LLAMA_ATTN_ERR_UNSUPPORTED;
+  const int Lmax = static_cast<int>(Lmax64);
+  if (!aligned16(kpages) || !aligned16(vpages) || !aligned16(q) || !aligned16(out)) return LLAMA_ATTN_ERR_INVALID_ARG;
+  const size_t need = llama_attn_decode_workspace_size(B, Hq, Lmax, D);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < need) return LLAMA_ATTN_ERR_WORKSPACE;
+  int dev, st;
+  if ((st = current_device(&dev))) return st;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceCache& dc = g_cache[dev];
+  const float2* tab = nullptr;
+  if ((st = rope_table(dc, static_cast<double>(rope_theta), D, Lmax + 1, stream, &tab))) return st;
+
+  CUtensorMap tk, tv;
+  const int64_t rows = static_cast<int64_t>(n_pages) * Hkv * page_size;
+  if ((st = tmap_rows(&tk, kpages, rows))) return st;
+  if ((st = tmap_rows(&tv, vpages, rows))) return st;
+
+  la::dec::Params p;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.Lmax = Lmax;
+  p.nchunk = (Lmax + la::dec::CHUNK - 1) / la::dec::CHUNK;
+  p.lens = cache_lens;
+  p.q = q;
+  p.rope_tab = reinterpret_cast<const float4*>(tab);
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  p.epoch = next_epoch();
+  p.rope_theta = static_cast<double>(rope_theta);
+  p.block_table = block_table;
+  p.page_size = page_size;
+  p.max_blocks = max_blocks;
+  p.n_pages = n_pages;
+  const size_t slots = static_cast<size_t>(B) * Hq * p.nchunk;
+  p.part_o = static_cast<float*>(workspace);
+  p.part_lse = p.part_o + slots * 128;
+  if (!dc.decode_paged_attr_set) {
+    LA_CUDA(cudaFuncSetAttribute(la::dec::decode_split_kernel<false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, la::dec::SMEM_ALLOC));
+    dc.decode_paged_attr_set = true;
+  }
+  const dim3 grid(p.nchunk, Hkv, B);
+  prof_count(2);
+  const int pair = prof_before(stream);
+  la::dec::decode_split_kernel<false, true><<<grid, la::dec::NTHREADS, la::dec::SMEM_ALLOC, stream>>>(tk, tv, p);
+  const cudaError_t e = cudaGetLastError();
+  prof_after(pair, stream);
+  if (e != cudaSuccess) return LLAMA_ATTN_ERR_CUDA;
   la::dec::decode_combine_kernel<<<B * Hq, 128, 0, stream>>>(p.part_o, p.part_lse, cache_lens, out, Hq, Lmax,
                                                             p.nchunk);
   return cuda_status(cudaGetLastError());

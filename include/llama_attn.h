@@ -148,6 +148,32 @@ int llama_attn_decode(const llama_attn_bf16 *q, const llama_attn_bf16 *kcache,
                       cudaStream_t stream);
 
 /*
+ * llama_attn_decode against a paged KV cache (block-table indirection, the
+ * dynamic KV-cache management named on the fifth page, "Meta's Llama 3 ...",
+ * serving paragraph): the cache of every sequence is a list of fixed-size
+ * pages in a shared pool.
+ *
+ *   kpages, vpages  [n_pages, Hkv, page_size, D] bf16: page p holds page_size
+ *                   consecutive cache rows of every KV head (keys already
+ *                   rotated at their positions)
+ *   block_table     [B, max_blocks] int32, device: logical block j of sequence
+ *                   b (cache rows j*page_size .. (j+1)*page_size - 1) is page
+ *                   block_table[b * max_blocks + j]; entries past the
+ *                   sequence's length are never read
+ *   cache_lens      [B] int32, device, 0 <= len <= max_blocks * page_size
+ *   page_size       a multiple of 64
+ * Everything else (q, out, rotation, workspace with Lmax = max_blocks *
+ * page_size, errors) is as in llama_attn_decode. A block id outside
+ * [0, n_pages) sets LLAMA_ATTN_DEVERR_BLOCK_TABLE and its rows read as zero.
+ */
+int llama_attn_decode_paged(const llama_attn_bf16 *q, const llama_attn_bf16 *kpages,
+                            const llama_attn_bf16 *vpages, const int32_t *block_table,
+                            const int32_t *cache_lens, llama_attn_bf16 *out, int B, int Hq,
+                            int Hkv, int D, int page_size, int max_blocks, int n_pages,
+                            float rope_theta, void *workspace, size_t workspace_bytes,
+                            cudaStream_t stream);
+
+/*
  * llama_attn_decode without a caller-supplied workspace and without any
  * device allocation, for callers that cannot allocate device memory: code
  * that runs inside a CUDA graph capture, under an allocator that owns all of
@@ -183,6 +209,7 @@ const char *llama_attn_status_string(int status);
 #define LLAMA_ATTN_DEVERR_TIMEOUT 0x1     /* a bounded wait on a barrier gave up */
 #define LLAMA_ATTN_DEVERR_DOC_OFFSETS 0x2 /* malformed doc_offsets */
 #define LLAMA_ATTN_DEVERR_CACHE_LEN 0x4   /* cache_lens[b] outside [0, Lmax] */
+#define LLAMA_ATTN_DEVERR_BLOCK_TABLE 0x8 /* a paged-cache block id outside [0, n_pages) */
 
 /*
  * Waits for `stream`, then returns and clears the current device's error word
