@@ -511,8 +511,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int c = 0; c < 128; c += 2) {
           float x0, x1;
           f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sl2x2, negmx2), x0, x1);
-          // one pair in four goes through the FMA-pipe polynomial, the rest through MUFU
-          const bool poly = (c & 6) == 6;
+          // one pair in eight goes through the FMA-pipe polynomial, the rest through
+          // MUFU (a larger share measured slower: it raises register pressure)
+          const bool poly = (c & 14) == 14;
           const float p0 = poly ? ex2_poly(x0) : ex2_approx(x0);
           const float p1 = poly ? ex2_poly(x1) : ex2_approx(x1);
           if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));

@@ -1,4 +1,4 @@
-"""The FMA-pipe 2^x used for a quarter of the softmax exponentials: its
+"""The FMA-pipe 2^x used for one softmax exponential in eight: its
 constants come from the committed fit, and the float32 evaluation (range
 reduction + cubic + exponent add) stays within 1e-4 relative error of exp2."""
 import os
