@@ -29,6 +29,7 @@ EXPORTED = (
     "llama_attn_decode_noalloc",
     "llama_attn_prefill_ex",
     "llama_attn_decode_paged",
+    "llama_attn_prefill_cp",
 )
 
 DEVERR_TIMEOUT = 0x1
@@ -78,6 +79,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.llama_attn_prefill_ex.restype = I
     lib.llama_attn_decode_paged.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, P, Z, P]
     lib.llama_attn_decode_paged.restype = I
+    lib.llama_attn_prefill_cp.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, P]
+    lib.llama_attn_prefill_cp.restype = I
     return lib
 
 
@@ -187,6 +190,31 @@ def llama_attn_prefill_ex(q, k, v, out=None, lse=None, doc_offsets=None, rope_th
     st = lib().llama_attn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(doc_offsets), B, S, Hq,
                                      Hkv, D, float(rope_theta), _ptr(kcache), _ptr(vcache), Lmax, _stream(stream))
     _check("llama_attn_prefill_ex", st)
+    return out, lse
+
+
+def llama_attn_prefill_cp(q, k, v, q_pos_a: int, q_split: int, q_pos_b: int = 0, out=None, lse=None,
+                          rope_theta: float = 500000.0, stream=None):
+    """bf16 prefill of query chunks against a whole sequence (one step of
+    context parallelism). q [B,Sq,Hq,D]: rows [0, q_split) sit at global
+    positions q_pos_a.., rows [q_split, Sq) at q_pos_b..; k/v [B,Skv,Hkv,D]
+    are the whole sequence. Returns (out, lse)."""
+    import torch
+    _require(q.dim() == 4 and k.dim() == 4 and v.dim() == 4, "q, k, v must be [B, S, H, D]")
+    for t in (q, k, v):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "bf16 contiguous CUDA tensors expected")
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    _require(k.shape == (B, Skv, Hkv, D) and v.shape == k.shape, "k and v must be [B, Skv, Hkv, D]")
+    if out is None:
+        out = torch.empty_like(q)
+    _require(out.shape == q.shape and out.dtype == torch.bfloat16 and out.is_contiguous(), "bad out")
+    if lse is not None:
+        _require(lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.shape == (B, Sq, Hq),
+                 "lse: float32 [B, Sq, Hq]")
+    st = lib().llama_attn_prefill_cp(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Skv, Hq, Hkv, D,
+                                     int(q_pos_a), int(q_split), int(q_pos_b), float(rope_theta), _stream(stream))
+    _check("llama_attn_prefill_cp", st)
     return out, lse
 
 

@@ -294,26 +294,40 @@ namespace {
 
 // bf16 prefill shared by llama_attn_prefill and llama_attn_prefill_ex: lse,
 // kcache and vcache may be null (no log-sum-exp output, no cache append).
+// Query chunks (context parallelism): q holds S rows per batch row, rows
+// [0, q_split) at global positions q_pos_a.., rows [q_split, S) at q_pos_b..;
+// k and v hold the whole sequence, Skv rows. A plain prefill is
+// Skv = q_split = S, q_pos_a = q_pos_b = 0.
+struct QChunks {
+  int Skv, q_split, q_pos_a, q_pos_b;
+};
+
 int prefill_bf16_impl(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
                       llama_attn_bf16* out, float* lse, const int32_t* doc_offsets, int B, int S, int Hq, int Hkv,
                       int D, float rope_theta, llama_attn_bf16* kcache, llama_attn_bf16* vcache, int Lmax,
-                      cudaStream_t stream) {
+                      const QChunks& qc, cudaStream_t stream) {
   int st = check_prefill_common(q, k, v, out, B, S, Hq, Hkv, rope_theta);
   if (st) return st;
+  const int Skv = qc.Skv;
+  if (Skv <= 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * Skv > INT32_MAX) return LLAMA_ATTN_ERR_UNSUPPORTED;
   if (D != 128) return LLAMA_ATTN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LLAMA_ATTN_ERR_INVALID_ARG;
   if ((kcache == nullptr) != (vcache == nullptr)) return LLAMA_ATTN_ERR_INVALID_ARG;
   if (kcache && (Lmax < S || !aligned16(kcache) || !aligned16(vcache))) return LLAMA_ATTN_ERR_INVALID_ARG;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LLAMA_ATTN_ERR_INVALID_ARG;
   if (static_cast<int64_t>(S) * Hq * 256 >= (int64_t(1) << 40)) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(Skv) * Hkv * 256 >= (int64_t(1) << 40)) return LLAMA_ATTN_ERR_UNSUPPORTED;
   int dev;
   if ((st = current_device(&dev))) return st;
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceCache& dc = g_cache[dev];
 
   const float2* tab = nullptr;
-  if ((st = rope_table(dc, static_cast<double>(rope_theta), D, S, stream, &tab))) return st;
+  const int n_pos = S > Skv ? S : Skv;
+  if ((st = rope_table(dc, static_cast<double>(rope_theta), D, n_pos, stream, &tab))) return st;
   const int64_t ntok = static_cast<int64_t>(B) * S;
+  const int64_t nkv_tok = static_cast<int64_t>(B) * Skv;
   const int32_t* doc_start = nullptr;
   if (doc_offsets) {
     if ((st = grow(reinterpret_cast<void**>(&dc.doc_start), &dc.doc_bytes, sizeof(int32_t) * ntok))) return st;
@@ -322,13 +336,14 @@ int prefill_bf16_impl(const llama_attn_bf16* q, const llama_attn_bf16* k, const 
     LA_CUDA(cudaGetLastError());
     doc_start = dc.doc_start;
   }
-  const size_t kbytes = static_cast<size_t>(ntok) * Hkv * 128 * 2;
+  const size_t kbytes = static_cast<size_t>(nkv_tok) * Hkv * 128 * 2;
   if ((st = grow(&dc.krot, &dc.krot_bytes, kbytes))) return st;
   const int64_t nvec = ntok * Hkv * 16;
+  const int64_t nvec_kv = nkv_tok * Hkv * 16;
   prof_count(1);
-  la::rope_rotate_rows_bf16_kernel<<<grid_for(nvec, 256), 256, 0, stream>>>(
+  la::rope_rotate_rows_bf16_kernel<<<grid_for(nvec_kv, 256), 256, 0, stream>>>(
       reinterpret_cast<const uint4*>(k), reinterpret_cast<uint4*>(dc.krot), reinterpret_cast<const float4*>(tab),
-      doc_start, S, Hkv, nvec);
+      doc_start, Skv, Hkv, nvec_kv);
   LA_CUDA(cudaGetLastError());
   if (kcache) {
     prof_count(1);
@@ -340,8 +355,8 @@ int prefill_bf16_impl(const llama_attn_bf16* q, const llama_attn_bf16* k, const 
 
   CUtensorMap tq, tk, tv, to;
   if ((st = tmap_bshd(&tq, q, B, S, Hq))) return st;
-  if ((st = tmap_bshd(&tk, dc.krot, B, S, Hkv))) return st;
-  if ((st = tmap_bshd(&tv, v, B, S, Hkv))) return st;
+  if ((st = tmap_bshd(&tk, dc.krot, B, Skv, Hkv))) return st;
+  if ((st = tmap_bshd(&tv, v, B, Skv, Hkv))) return st;
   if ((st = tmap_bshd(&to, out, B, S, Hq))) return st;
 
   la::pfx::Params p;
@@ -353,6 +368,11 @@ int prefill_bf16_impl(const llama_attn_bf16* q, const llama_attn_bf16* k, const 
   p.NH = (p.G % 2 == 0) ? 2 : 1;
   p.n_qt = (S + la::pfx::BM - 1) / la::pfx::BM;
   p.n_hp = Hq / p.NH;
+  p.Skv = Skv;
+  p.n_pos = n_pos;
+  p.q_split = qc.q_split;
+  p.q_pos_a = qc.q_pos_a;
+  p.q_pos_b = qc.q_pos_b;
   p.doc_start = doc_start;
   p.rope_tab = reinterpret_cast<const float4*>(tab);
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
@@ -387,7 +407,7 @@ int llama_attn_prefill(const llama_attn_bf16* q, const llama_attn_bf16* k, const
                        llama_attn_bf16* out, const int32_t* doc_offsets, int B, int S, int Hq, int Hkv, int D,
                        float rope_theta, cudaStream_t stream) {
   return prefill_bf16_impl(q, k, v, out, nullptr, doc_offsets, B, S, Hq, Hkv, D, rope_theta, nullptr, nullptr, 0,
-                           stream);
+                           QChunks{S, S, 0, 0}, stream);
 }
 
 int llama_attn_prefill_ex(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
@@ -395,7 +415,20 @@ int llama_attn_prefill_ex(const llama_attn_bf16* q, const llama_attn_bf16* k, co
                           int Hkv, int D, float rope_theta, llama_attn_bf16* kcache, llama_attn_bf16* vcache,
                           int Lmax, cudaStream_t stream) {
   return prefill_bf16_impl(q, k, v, out, lse, doc_offsets, B, S, Hq, Hkv, D, rope_theta, kcache, vcache, Lmax,
-                           stream);
+                           QChunks{S, S, 0, 0}, stream);
+}
+
+int llama_attn_prefill_cp(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
+                          llama_attn_bf16* out, float* lse, int B, int Sq, int Skv, int Hq, int Hkv, int D,
+                          int q_pos_a, int q_split, int q_pos_b, float rope_theta, cudaStream_t stream) {
+  if (B <= 0 || Sq <= 0 || Skv <= 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  constexpr int kT = la::pfx::BM;
+  if (q_split < 0 || q_split > Sq || q_pos_a < 0 || q_pos_b < 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (q_split % kT != 0 || q_pos_a % kT != 0 || q_pos_b % kT != 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(q_pos_a) + q_split > Skv) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(q_pos_b) + (Sq - q_split) > Skv) return LLAMA_ATTN_ERR_INVALID_ARG;
+  return prefill_bf16_impl(q, k, v, out, lse, nullptr, B, Sq, Hq, Hkv, D, rope_theta, nullptr, nullptr, 0,
+                           QChunks{Skv, q_split, q_pos_a, q_pos_b}, stream);
 }
 
 int llama_attn_prefill_f32(const float* q, const float* k, const float* v, float* out, const int32_t* doc_offsets,

@@ -79,6 +79,12 @@ static_assert(N_BARS * 8 + 8 + 8 * kItemRing <= 512, "barrier area, TMEM address
 
 struct Params {
   int B, S, Hq, Hkv, G, NH, n_qt, n_hp;
+  // Key/value rows per batch row (S unless the queries are chunks of a longer
+  // sequence) and RoPE table rows (max(S, Skv)).
+  int Skv, n_pos;
+  // Global position of local query row 0 and of local row q_split (a multiple
+  // of 128; S when all rows form one chunk). Both 0 for a plain prefill.
+  int q_split, q_pos_a, q_pos_b;
   const int32_t* doc_start;  // [B*S] row-local document start, or null (one document per row)
   const float4* rope_tab;    // (cos, sin) pairs, 64 per position, as float4 = 2 pairs
   int* sched;                // work-item counter, zero at launch
@@ -98,6 +104,11 @@ struct Item {
   int64_t rowbase;
 };
 
+// Global position of local query row q0 (a multiple of 128).
+__device__ __forceinline__ int q_global(int q0, const Params& p) {
+  return (q0 < p.q_split) ? p.q_pos_a + q0 : p.q_pos_b + (q0 - p.q_split);
+}
+
 __device__ __forceinline__ Item item_of(int item, const Params& p) {
   Item it;
   const int per_rank = p.B * p.n_hp;
@@ -112,7 +123,7 @@ __device__ __forceinline__ Item item_of(int item, const Params& p) {
   const int ds_first = p.doc_start ? p.doc_start[it.rowbase + it.q0] : 0;
   it.ds_last = p.doc_start ? p.doc_start[it.rowbase + q_last] : 0;
   it.kv_t0 = ds_first / BN;
-  it.n_kv = qt - it.kv_t0 + 1;
+  it.n_kv = q_global(it.q0, p) / BN - it.kv_t0 + 1;  // the last tile holds the diagonal
   return it;
 }
 
@@ -202,10 +213,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (v < 0 || v >= n_items) return;
         const Item J = item_of(v, p);
         const int ds0 = p.doc_start ? p.doc_start[J.rowbase + J.q0] : 0;
-        const int p0 = J.q0 - ds0;
-        const int n0 = min(BM, p.S - p0);
+        const int p0 = q_global(J.q0, p) - ds0;
+        const int n0 = min(BM, p.n_pos - p0);
         if (n0 > 0) bulk_prefetch_l2(p.rope_tab + static_cast<int64_t>(p0) * 32, static_cast<uint32_t>(n0) * 512u);
-        if (J.ds_last > J.q0) bulk_prefetch_l2(p.rope_tab, static_cast<uint32_t>(min(BM, p.S)) * 512u);
+        if (J.ds_last > J.q0) bulk_prefetch_l2(p.rope_tab, static_cast<uint32_t>(min(BM, p.n_pos)) * 512u);
       };
       auto publish = [&](int k, int v) {
         ring_item[k % kItemRing] = v;
@@ -368,7 +379,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bool ok = true;
     uint32_t tiles = 0;
     Item I;
-    int qi_c = 0, ds_i = 0;
+    int qi_c = 0, ds_i = 0;  // global position of this thread's (clamped) row; its document start
     // Starts item `it`: reads its id from the ring, loads its row data, waits for
     // its Q tile and rotates this thread's row in place. False at the end of the
     // items (or on a timeout, which also clears ok).
@@ -403,6 +414,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int qi = I.q0 + r;
       qi_c = min(qi, p.S - 1);
       ds_i = p.doc_start ? p.doc_start[I.rowbase + qi_c] : 0;
+      qi_c += q_global(I.q0, p) - I.q0;  // from here on the row's global position
       if (!mbar_wait(bar(B_Q_FULL), it & 1, wc)) {
         ok = false;
         return false;
@@ -476,7 +488,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float sv[128];
 #pragma unroll
         for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c]);
-        if (kb + BN - 1 > I.q0 || kb < I.ds_last) {
+        if (j == I.n_kv - 1 || kb < I.ds_last) {  // the diagonal tile, or a document starts in it
           const int lo = ds_i - kb, hi = qi_c - kb;
 #pragma unroll
           for (int c = 0; c < 128; ++c) sv[c] = (c < lo || c > hi) ? -INFINITY : sv[c];

@@ -109,6 +109,36 @@ int llama_attn_prefill_ex(const llama_attn_bf16 *q, const llama_attn_bf16 *k,
                           int Lmax, cudaStream_t stream);
 
 /*
+ * Prefill of query chunks against a whole sequence: the per-GPU step of
+ * context parallelism ("Llama 3.1 Architecture: Dense Scaling to 405B and
+ * 128K Context", "The 4D Parallelism Execution Strategy", context-parallel
+ * bullet: the 128K sequence is split along tokens across GPUs and the KV
+ * states are exchanged). Each rank holds some query rows and, after an
+ * exchange of keys and values, the whole sequence's k and v; this call
+ * computes causal attention of its query rows over that sequence.
+ *
+ *   q   [B, Sq, Hq, D]  un-rotated queries: local rows [0, q_split) are the
+ *                       tokens at global positions q_pos_a .. q_pos_a+q_split-1,
+ *                       rows [q_split, Sq) those at q_pos_b .. q_pos_b+Sq-q_split-1
+ *   k   [B, Skv, Hkv, D] un-rotated keys of the whole sequence (positions 0..Skv-1)
+ *   v   [B, Skv, Hkv, D] values of the whole sequence
+ *   out [B, Sq, Hq, D]  result for the local query rows
+ *   lse [B, Sq, Hq] float32, or NULL: as for llama_attn_prefill_ex
+ *
+ * Each batch row is one document (no cross-document mask); the query at global
+ * position P sees keys 0..P and is rotated at P. q_split, q_pos_a and q_pos_b
+ * are multiples of 128 (the kernel's query tile), 0 <= q_split <= Sq,
+ * q_pos_a + q_split <= Skv and q_pos_b + (Sq - q_split) <= Skv; otherwise
+ * LLAMA_ATTN_ERR_INVALID_ARG. With Skv = Sq = q_split and q_pos_a = 0 the
+ * result equals llama_attn_prefill with doc_offsets NULL. Other errors and the
+ * scratch (a rotated copy of the Skv keys) as for llama_attn_prefill.
+ */
+int llama_attn_prefill_cp(const llama_attn_bf16 *q, const llama_attn_bf16 *k,
+                          const llama_attn_bf16 *v, llama_attn_bf16 *out, float *lse, int B,
+                          int Sq, int Skv, int Hq, int Hkv, int D, int q_pos_a, int q_split,
+                          int q_pos_b, float rope_theta, cudaStream_t stream);
+
+/*
  * Prefill in true fp32 arithmetic on CUDA cores (FFMA, accurate expf), same
  * semantics and layouts as llama_attn_prefill with float tensors.
  * D even, 2 <= D <= 128.
