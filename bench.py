@@ -326,6 +326,116 @@ def run_ours(args, w):
         dist.destroy_process_group()
 
 
+def run_cp(args, w):
+    """Context-parallel prefill of one workload over the ranks (strong
+    scaling): every rank holds its zigzag shard of q, k and v; a step is the
+    K/V all-gather plus the local llama_attn_prefill_cp call."""
+    import gqa_attention_rope_b200 as la
+    from gqa_attention_rope_b200 import context_parallel as CP
+    if w.doc_range is not None:
+        raise SystemExit("--cp takes a single-document workload (each batch row one document)")
+    world, rank, local = dist_setup(args.gpus)
+    group = None
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    la.lib()
+    hbm_peak, tc_peak, tc_sust, peak_kind = load_peaks()
+    inp = W.make_prefill_inputs(w)  # the same seeded sequence on every rank
+    ql, kl, vl = (CP.shard_rows(inp[n], world, rank).to(dev) for n in ("q", "k", "v"))
+    pos_a, pos_b, L = CP.zigzag_chunks(w.S, world, rank)
+    rows = np.r_[pos_a:pos_a + L, pos_b:pos_b + L]
+    flops_local = 4.0 * w.D * w.Hq * w.B * float(np.sum(rows + 1))
+    flops_total = 4.0 * w.D * w.Hq * W.unmasked_pairs(None, w.B, w.S)
+    out = torch.empty_like(ql)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(q_, k_, v_, o_):
+        k_full = CP.gather_sequence(k_, world, group)
+        v_full = CP.gather_sequence(v_, world, group)
+        la.llama_attn_prefill_cp(q_, k_full, v_full, pos_a, L, pos_b, out=o_, rope_theta=w.rope_theta)
+
+    for _ in range(max(3, args.warmup)):
+        step(ql, kl, vl, out)
+    torch.cuda.synchronize()
+    if la.llama_attn_get_device_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    la.llama_attn_profile_begin()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step(ql, kl, vl, out)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    main_ms, main_n, launches = la.llama_attn_profile_end()
+    barrier(world)
+    clk = clocks.stop()
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), world)
+    value = flops_total * args.steps / (total_ms / 1e3) / 1e12
+    kernel_ms = main_ms / max(main_n, 1)
+    achieved = flops_local / (kernel_ms / 1e3) / 1e12
+
+    # end to end: the rank's pinned host shards in, its output rows back
+    hq, hk, hv = (t.cpu().pin_memory() for t in (ql, kl, vl))
+    hout = torch.empty(ql.shape, dtype=ql.dtype).pin_memory()
+    dq, dk, dv, dout = torch.empty_like(ql), torch.empty_like(kl), torch.empty_like(vl), torch.empty_like(ql)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        step(dq, dk, dv, dout)
+        hout.copy_(dout, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    for i in range(args.steps):
+        e_ev[i][0].record(stream)
+        e2e_step()
+        e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev), world)
+    if la.llama_attn_get_device_error() != 0:
+        raise RuntimeError("device error word set during the benchmark")
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, s, n, threads = oracle_rows_sample(w, inp, args.cpu_seconds)
+        cpu = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n} random query rows x {w.Hq} heads of {w.name} (float64 C oracle, "
+                         f"full masked rows, {s:.1f} s)"}
+    cfg = config_of(w, world)
+    cfg["parallelism"] = (f"context parallel over {world} GPU(s): zigzag split into {2 * world} chunks, "
+                          "K/V all-gather (NCCL) into local memory, local kernel")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(cfg, flops_per_step_total=flops_total),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
+                     "frac": achieved / tc_peak, "peak_kind": f"{peak_kind} bf16 dense (burst)",
+                     "kernel": "prefill_bf16_kernel", "kernel_ms": kernel_ms, "traffic": None},
+        "cpu_baseline": cpu,
+        "e2e": {"value": flops_total * args.steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hq, hk, hv)),
+                "d2h_bytes_per_step": hout.numel() * hout.element_size()},
+        "clocks": clk,
+        "gpu_launches": launches,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def run_decode(args, la, dev, world, rank, hbm_peak, peak_kind):
     w = W.DECODE_70B
     nseq = args.decode_seqs
@@ -440,6 +550,8 @@ def main():
     ap.add_argument("--decode-page-size", type=int, default=0,
                     help="time the decode through the paged-cache entry point with this page size")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cp", action="store_true",
+                    help="context-parallel prefill of the workload over the GPUs (strong scaling)")
     args = ap.parse_args()
     w = W.WORKLOADS[args.workload]
     if args.impl == "reference":
@@ -447,7 +559,7 @@ def main():
     else:
         if w.dtype != "bf16":
             raise SystemExit("the bench times the bf16 tensor-core path")
-        run_ours(args, w)
+        run_cp(args, w) if args.cp else run_ours(args, w)
 
 
 if __name__ == "__main__":
