@@ -30,6 +30,9 @@ EXPORTED = (
     "llama_attn_prefill_ex",
     "llama_attn_decode_paged",
     "llama_attn_prefill_cp",
+    "llama_attn_prefill_rotated",
+    "llama_attn_quantize_e4m3",
+    "llama_attn_qkv_fp8_rope",
 )
 
 DEVERR_TIMEOUT = 0x1
@@ -81,6 +84,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.llama_attn_decode_paged.restype = I
     lib.llama_attn_prefill_cp.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, I, F, P]
     lib.llama_attn_prefill_cp.restype = I
+    lib.llama_attn_prefill_rotated.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P]
+    lib.llama_attn_prefill_rotated.restype = I
+    lib.llama_attn_quantize_e4m3.argtypes = [P, ctypes.c_int64, P, P, P]
+    lib.llama_attn_quantize_e4m3.restype = I
+    lib.llama_attn_qkv_fp8_rope.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.llama_attn_qkv_fp8_rope.restype = I
     return lib
 
 
@@ -216,6 +225,75 @@ def llama_attn_prefill_cp(q, k, v, q_pos_a: int, q_split: int, q_pos_b: int = 0,
                                      int(q_pos_a), int(q_split), int(q_pos_b), float(rope_theta), _stream(stream))
     _check("llama_attn_prefill_cp", st)
     return out, lse
+
+
+def llama_attn_prefill_rotated(q, k, v, out=None, lse=None, doc_offsets=None, stream=None):
+    """bf16 prefill on already-rotated q [B,S,Hq,D] and k [B,S,Hkv,D] (no RoPE
+    step). Returns (out, lse)."""
+    import torch
+    _require(q.dim() == 4 and k.dim() == 4 and v.dim() == 4, "q, k, v must be [B, S, H, D]")
+    for t in (q, k, v):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "bf16 contiguous CUDA tensors expected")
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _require(k.shape == (B, S, Hkv, D) and v.shape == k.shape, "k and v must be [B, S, Hkv, D]")
+    if out is None:
+        out = torch.empty_like(q)
+    _require(out.shape == q.shape and out.dtype == torch.bfloat16 and out.is_contiguous(), "bad out")
+    if lse is not None:
+        _require(lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.shape == (B, S, Hq),
+                 "lse: float32 [B, S, Hq]")
+    if doc_offsets is not None:
+        _require(doc_offsets.is_cuda and doc_offsets.dtype == torch.int32, "doc_offsets: int32 CUDA tensor")
+    st = lib().llama_attn_prefill_rotated(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(doc_offsets), B, S,
+                                          Hq, Hkv, D, _stream(stream))
+    _check("llama_attn_prefill_rotated", st)
+    return out, lse
+
+
+def llama_attn_quantize_e4m3(x, y=None, scale=None, stream=None):
+    """Per-tensor dynamic E4M3 quantization of a bf16 CUDA tensor. Returns
+    (codes uint8 tensor of x's shape, scale float32 CUDA tensor of one element)."""
+    import torch
+    _require(x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous(), "x: bf16 contiguous CUDA tensor")
+    if y is None:
+        y = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty(1, dtype=torch.float32, device=x.device)
+    _require(y.is_cuda and y.dtype == torch.uint8 and y.is_contiguous() and y.numel() == x.numel(), "bad y")
+    _require(scale.is_cuda and scale.dtype == torch.float32 and scale.numel() >= 1, "bad scale")
+    st = lib().llama_attn_quantize_e4m3(_ptr(x), x.numel(), _ptr(y), _ptr(scale), _stream(stream))
+    _check("llama_attn_quantize_e4m3", st)
+    return y, scale
+
+
+def llama_attn_qkv_fp8_rope(x, s_x, w, s_w, B: int, S: int, Hq: int, Hkv: int, doc_offsets=None,
+                            rope_theta: float = 500000.0, q=None, k=None, v=None, stream=None):
+    """FP8 QKV projection with RoPE. x [B*S, d_model] and w [(Hq+2Hkv)*128,
+    d_model] are uint8 E4M3 codes, s_x / s_w one-element float32 CUDA tensors.
+    Returns (q rotated [B,S,Hq,128], k rotated [B,S,Hkv,128], v [B,S,Hkv,128]) bf16."""
+    import torch
+    D = 128
+    for t in (x, w):
+        _require(t.is_cuda and t.dtype == torch.uint8 and t.is_contiguous() and t.dim() == 2, "uint8 2-D codes")
+    d_model = x.shape[1]
+    _require(x.shape[0] == B * S and w.shape == ((Hq + 2 * Hkv) * D, d_model), "x / w shapes")
+    for t in (s_x, s_w):
+        _require(t.is_cuda and t.dtype == torch.float32, "scales: float32 CUDA tensors")
+    dev = x.device
+    if q is None:
+        q = torch.empty(B, S, Hq, D, dtype=torch.bfloat16, device=dev)
+    if k is None:
+        k = torch.empty(B, S, Hkv, D, dtype=torch.bfloat16, device=dev)
+    if v is None:
+        v = torch.empty(B, S, Hkv, D, dtype=torch.bfloat16, device=dev)
+    if doc_offsets is not None:
+        _require(doc_offsets.is_cuda and doc_offsets.dtype == torch.int32, "doc_offsets: int32 CUDA tensor")
+    st = lib().llama_attn_qkv_fp8_rope(_ptr(x), _ptr(s_x), _ptr(w), _ptr(s_w), _ptr(q), _ptr(k), _ptr(v),
+                                       _ptr(doc_offsets), B, S, d_model, Hq, Hkv, D, float(rope_theta),
+                                       _stream(stream))
+    _check("llama_attn_qkv_fp8_rope", st)
+    return q, k, v
 
 
 def llama_attn_prefill_f32(q, k, v, out=None, doc_offsets=None, rope_theta: float = 500000.0, stream=None):

@@ -13,6 +13,7 @@
 #include "rope.cuh"
 #include "prefill_f32.cuh"
 #include "prefill_bf16.cuh"
+#include "qkv_fp8.cuh"
 #include "decode.cuh"
 
 #define LLAMA_ATTN_VERSION 100  // 0.1.0
@@ -38,6 +39,8 @@ struct DeviceCache {
   bool prefill_attr_set = false;
   bool decode_attr_set = false;
   bool decode_paged_attr_set = false;
+  unsigned int* amax = nullptr;  // per-tensor amax of the E4M3 quantizer
+  bool qkv_attr_set = false;
 };
 
 std::mutex g_mutex;
@@ -206,6 +209,22 @@ int tmap_rows(CUtensorMap* map, const void* ptr, int64_t rows) {
   return r == CUDA_SUCCESS ? LLAMA_ATTN_OK : LLAMA_ATTN_ERR_CUDA;
 }
 
+// Row-major [rows, cols] matrix of 1- or 2-byte elements as a 2-D tensor map
+// (cols innermost), box box_cols x box_rows, 128-byte swizzle (box_cols *
+// elem_bytes == 128). Rows past `rows` read as zero and are not written.
+int tmap_2d(CUtensorMap* map, const void* ptr, CUtensorMapDataType dt, int elem_bytes, int64_t rows, int64_t cols,
+            int box_cols, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return LLAMA_ATTN_ERR_CUDA;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * elem_bytes};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LLAMA_ATTN_OK : LLAMA_ATTN_ERR_CUDA;
+}
+
 int check_prefill_common(const void* q, const void* k, const void* v, const void* out, int B, int S, int Hq,
                          int Hkv, float rope_theta) {
   if (!q || !k || !v || !out) return LLAMA_ATTN_ERR_INVALID_ARG;
@@ -305,7 +324,7 @@ struct QChunks {
 int prefill_bf16_impl(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
                       llama_attn_bf16* out, float* lse, const int32_t* doc_offsets, int B, int S, int Hq, int Hkv,
                       int D, float rope_theta, llama_attn_bf16* kcache, llama_attn_bf16* vcache, int Lmax,
-                      const QChunks& qc, cudaStream_t stream) {
+                      const QChunks& qc, cudaStream_t stream, bool prerotated = false) {
   int st = check_prefill_common(q, k, v, out, B, S, Hq, Hkv, rope_theta);
   if (st) return st;
   const int Skv = qc.Skv;
@@ -325,7 +344,7 @@ int prefill_bf16_impl(const llama_attn_bf16* q, const llama_attn_bf16* k, const 
 
   const float2* tab = nullptr;
   const int n_pos = S > Skv ? S : Skv;
-  if ((st = rope_table(dc, static_cast<double>(rope_theta), D, n_pos, stream, &tab))) return st;
+  if (!prerotated && (st = rope_table(dc, static_cast<double>(rope_theta), D, n_pos, stream, &tab))) return st;
   const int64_t ntok = static_cast<int64_t>(B) * S;
   const int64_t nkv_tok = static_cast<int64_t>(B) * Skv;
   const int32_t* doc_start = nullptr;
@@ -337,14 +356,18 @@ int prefill_bf16_impl(const llama_attn_bf16* q, const llama_attn_bf16* k, const 
     doc_start = dc.doc_start;
   }
   const size_t kbytes = static_cast<size_t>(nkv_tok) * Hkv * 128 * 2;
-  if ((st = grow(&dc.krot, &dc.krot_bytes, kbytes))) return st;
+  if (!prerotated && (st = grow(&dc.krot, &dc.krot_bytes, kbytes))) return st;
   const int64_t nvec = ntok * Hkv * 16;
   const int64_t nvec_kv = nkv_tok * Hkv * 16;
-  prof_count(1);
-  la::rope_rotate_rows_bf16_kernel<<<grid_for(nvec_kv, 256), 256, 0, stream>>>(
-      reinterpret_cast<const uint4*>(k), reinterpret_cast<uint4*>(dc.krot), reinterpret_cast<const float4*>(tab),
-      doc_start, Skv, Hkv, nvec_kv);
-  LA_CUDA(cudaGetLastError());
+  const void* k_rot = k;  // pre-rotated keys are read as given
+  if (!prerotated) {
+    prof_count(1);
+    la::rope_rotate_rows_bf16_kernel<<<grid_for(nvec_kv, 256), 256, 0, stream>>>(
+        reinterpret_cast<const uint4*>(k), reinterpret_cast<uint4*>(dc.krot), reinterpret_cast<const float4*>(tab),
+        doc_start, Skv, Hkv, nvec_kv);
+    LA_CUDA(cudaGetLastError());
+    k_rot = dc.krot;
+  }
   if (kcache) {
     prof_count(1);
     la::kv_cache_append_kernel<<<grid_for(nvec, 256), 256, 0, stream>>>(
@@ -355,7 +378,7 @@ int prefill_bf16_impl(const llama_attn_bf16* q, const llama_attn_bf16* k, const 
 
   CUtensorMap tq, tk, tv, to;
   if ((st = tmap_bshd(&tq, q, B, S, Hq))) return st;
-  if ((st = tmap_bshd(&tk, dc.krot, B, Skv, Hkv))) return st;
+  if ((st = tmap_bshd(&tk, k_rot, B, Skv, Hkv))) return st;
   if ((st = tmap_bshd(&tv, v, B, Skv, Hkv))) return st;
   if ((st = tmap_bshd(&to, out, B, S, Hq))) return st;
 
@@ -373,6 +396,7 @@ int prefill_bf16_impl(const llama_attn_bf16* q, const llama_attn_bf16* k, const 
   p.q_split = qc.q_split;
   p.q_pos_a = qc.q_pos_a;
   p.q_pos_b = qc.q_pos_b;
+  p.q_rotated = prerotated ? 1 : 0;
   p.doc_start = doc_start;
   p.rope_tab = reinterpret_cast<const float4*>(tab);
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
@@ -429,6 +453,106 @@ int llama_attn_prefill_cp(const llama_attn_bf16* q, const llama_attn_bf16* k, co
   if (static_cast<int64_t>(q_pos_b) + (Sq - q_split) > Skv) return LLAMA_ATTN_ERR_INVALID_ARG;
   return prefill_bf16_impl(q, k, v, out, lse, nullptr, B, Sq, Hq, Hkv, D, rope_theta, nullptr, nullptr, 0,
                            QChunks{Skv, q_split, q_pos_a, q_pos_b}, stream);
+}
+
+int llama_attn_prefill_rotated(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
+                               llama_attn_bf16* out, float* lse, const int32_t* doc_offsets, int B, int S, int Hq,
+                               int Hkv, int D, cudaStream_t stream) {
+  return prefill_bf16_impl(q, k, v, out, lse, doc_offsets, B, S, Hq, Hkv, D, 500000.f, nullptr, nullptr, 0,
+                           QChunks{S, S, 0, 0}, stream, true);
+}
+
+int llama_attn_quantize_e4m3(const llama_attn_bf16* x, int64_t n, uint8_t* y, float* scale, cudaStream_t stream) {
+  if (!x || !y || !scale || n <= 0 || n % 8 != 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(y) & 7u) || (reinterpret_cast<uintptr_t>(scale) & 3u))
+    return LLAMA_ATTN_ERR_INVALID_ARG;
+  int dev, st;
+  if ((st = current_device(&dev))) return st;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceCache& dc = g_cache[dev];
+  if (dc.amax == nullptr) LA_CUDA(cudaMalloc(&dc.amax, 256));
+  LA_CUDA(cudaMemsetAsync(dc.amax, 0, sizeof(unsigned int), stream));
+  const int64_t nvec = n / 8;
+  int n_sm = 148;
+  if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
+  int64_t g = (nvec + 255) / 256;
+  const int grid = static_cast<int>(g < 4 * n_sm ? g : 4 * n_sm);
+  prof_count(2);
+  la::q8::amax_bf16_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), nvec, dc.amax);
+  LA_CUDA(cudaGetLastError());
+  la::q8::quantize_e4m3_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), nvec, dc.amax,
+                                                           reinterpret_cast<uint2*>(y), scale);
+  return cuda_status(cudaGetLastError());
+}
+
+int llama_attn_qkv_fp8_rope(const uint8_t* x, const float* s_x, const uint8_t* w, const float* s_w,
+                            llama_attn_bf16* q, llama_attn_bf16* k, llama_attn_bf16* v, const int32_t* doc_offsets,
+                            int B, int S, int d_model, int Hq, int Hkv, int D, float rope_theta,
+                            cudaStream_t stream) {
+  if (!x || !s_x || !w || !s_w || !q || !k || !v) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || S <= 0 || d_model <= 0 || Hq <= 0 || Hkv <= 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.f) || !std::isfinite(rope_theta)) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (D != 128 || d_model % la::q8::BK != 0) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(q) || !aligned16(k) || !aligned16(v)) return LLAMA_ATTN_ERR_INVALID_ARG;
+  const int64_t M = static_cast<int64_t>(B) * S;
+  const int64_t n_heads = static_cast<int64_t>(Hq) + 2 * Hkv;
+  if (M > INT32_MAX - 1 || n_heads * 128 > INT32_MAX || static_cast<int64_t>(Hq) * 256 >= (int64_t(1) << 32))
+    return LLAMA_ATTN_ERR_UNSUPPORTED;
+  int dev, st;
+  if ((st = current_device(&dev))) return st;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceCache& dc = g_cache[dev];
+  const float2* tab = nullptr;
+  if ((st = rope_table(dc, static_cast<double>(rope_theta), D, S, stream, &tab))) return st;
+  const int32_t* doc_start = nullptr;
+  if (doc_offsets) {
+    if ((st = grow(reinterpret_cast<void**>(&dc.doc_start), &dc.doc_bytes, sizeof(int32_t) * M))) return st;
+    prof_count(1);
+    la::doc_prep_kernel<<<1, 1024, 0, stream>>>(doc_offsets, B, S, dc.doc_start);
+    LA_CUDA(cudaGetLastError());
+    doc_start = dc.doc_start;
+  }
+  const int N = static_cast<int>(n_heads * 128);
+  CUtensorMap tx, tw, tq, tk, tv;
+  if ((st = tmap_2d(&tx, x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, M, d_model, la::q8::BK, la::q8::BM))) return st;
+  if ((st = tmap_2d(&tw, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, d_model, la::q8::BK, la::q8::BN))) return st;
+  if ((st = tmap_2d(&tq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, static_cast<int64_t>(Hq) * 128, 64, la::q8::BM)))
+    return st;
+  if ((st = tmap_2d(&tk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, static_cast<int64_t>(Hkv) * 128, 64, la::q8::BM)))
+    return st;
+  if ((st = tmap_2d(&tv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, M, static_cast<int64_t>(Hkv) * 128, 64, la::q8::BM)))
+    return st;
+  la::q8::Params p;
+  p.M = static_cast<int>(M);
+  p.K = d_model;
+  p.N = N;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.S = S;
+  p.n_mt = static_cast<int>((M + la::q8::BM - 1) / la::q8::BM);
+  p.n_nt = (N + la::q8::BN - 1) / la::q8::BN;
+  p.n_kb = d_model / la::q8::BK;
+  p.doc_start = doc_start;
+  p.rope_tab = reinterpret_cast<const float4*>(tab);
+  p.s_x = s_x;
+  p.s_w = s_w;
+  p.epoch = next_epoch();
+  const int64_t tiles = static_cast<int64_t>(p.n_mt) * p.n_nt;
+  if (tiles > INT32_MAX) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  if (!dc.qkv_attr_set) {
+    LA_CUDA(cudaFuncSetAttribute(la::q8::qkv_fp8_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 la::q8::SMEM_ALLOC));
+    dc.qkv_attr_set = true;
+  }
+  int n_sm = 148;
+  if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
+  const int grid = static_cast<int>(tiles < n_sm ? tiles : n_sm);
+  prof_count(1);
+  const int pair = prof_before(stream);
+  la::q8::qkv_fp8_rope_kernel<<<grid, la::q8::NTHREADS, la::q8::SMEM_ALLOC, stream>>>(tx, tw, tq, tk, tv, p);
+  const cudaError_t e = cudaGetLastError();
+  prof_after(pair, stream);
+  return cuda_status(e);
 }
 
 int llama_attn_prefill_f32(const float* q, const float* k, const float* v, float* out, const int32_t* doc_offsets,

@@ -85,6 +85,7 @@ struct Params {
   // Global position of local query row 0 and of local row q_split (a multiple
   // of 128; S when all rows form one chunk). Both 0 for a plain prefill.
   int q_split, q_pos_a, q_pos_b;
+  int q_rotated;             // 1: q arrives already rotated (no in-kernel rotation, no table)
   const int32_t* doc_start;  // [B*S] row-local document start, or null (one document per row)
   const float4* rope_tab;    // (cos, sin) pairs, 64 per position, as float4 = 2 pairs
   int* sched;                // work-item counter, zero at launch
@@ -210,7 +211,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // The RoPE table rows an item's Q rotation will read: positions
       // q0 - ds(q0) .. +127 and, when a document starts inside the tile, 0 .. 127.
       auto prefetch_rows = [&](int v) {
-        if (v < 0 || v >= n_items) return;
+        if (v < 0 || v >= n_items || p.q_rotated) return;
         const Item J = item_of(v, p);
         const int ds0 = p.doc_start ? p.doc_start[J.rowbase + J.q0] : 0;
         const int p0 = q_global(J.q0, p) - ds0;
@@ -425,7 +426,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // from the current ones by one rotation by 2*theta_k (angle addition,
       // the table's row for position 2). The table is read only for the first
       // row and where positions restart at a document start.
-      {
+      if (!p.q_rotated) {
         const int ch = lane & 15;
         const float4* step = p.rope_tab + 2 * 32 + 2 * ch;
         const float4 st0 = __ldg(step), st1 = __ldg(step + 1);

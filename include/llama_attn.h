@@ -139,6 +139,62 @@ int llama_attn_prefill_cp(const llama_attn_bf16 *q, const llama_attn_bf16 *k,
                           int q_pos_b, float rope_theta, cudaStream_t stream);
 
 /*
+ * Prefill on queries and keys that are already rotated (for example by
+ * llama_attn_qkv_fp8_rope): the same attention as llama_attn_prefill_ex
+ * without the RoPE step, so no rotated copy of k is made and no RoPE table
+ * is read. q [B, S, Hq, D] and k [B, S, Hkv, D] hold the rotated rows; v,
+ * out, lse, doc_offsets and the errors as for llama_attn_prefill_ex (no KV
+ * cache output). D == 128.
+ */
+int llama_attn_prefill_rotated(const llama_attn_bf16 *q, const llama_attn_bf16 *k,
+                               const llama_attn_bf16 *v, llama_attn_bf16 *out, float *lse,
+                               const int32_t *doc_offsets, int B, int S, int Hq, int Hkv, int D,
+                               cudaStream_t stream);
+
+/*
+ * Per-tensor dynamic E4M3 quantization ("Llama 3.1 Architecture: Dense
+ * Scaling to 405B and 128K Context", "FP8 Quantization: Fitting 405B on an
+ * 8xH100 Node": E4M3 with values up to 448, X_fp8 = clip(round(X / s_X),
+ * -448, 448) with one scale per tensor).
+ *
+ *   x      [n] bf16 (device, 16-byte aligned), n > 0 and n % 8 == 0
+ *   y      [n] E4M3 codes (device, 8-byte aligned): y_i = E4M3(x_i / s),
+ *          x_i / s an IEEE float32 division, rounded to nearest-even onto
+ *          the E4M3 grid and saturated to +-448
+ *   scale  one float (device): s = amax_i |x_i| / 448 in float32, or 1 when
+ *          x is all zeros
+ * The scale is left on the device, so a following llama_attn_qkv_fp8_rope
+ * reads it without a host round trip. NaN inputs give unspecified codes. The
+ * library keeps a 4-byte amax in per-device scratch.
+ */
+int llama_attn_quantize_e4m3(const llama_attn_bf16 *x, int64_t n, uint8_t *y, float *scale,
+                             cudaStream_t stream);
+
+/*
+ * FP8 QKV projection with RoPE: Y = (s_x * s_w) * (X_fp8 . W_fp8^T) on the
+ * tcgen05 tensor cores (E4M3 x E4M3, fp32 accumulation), split into the query,
+ * key and value heads, the query and key heads rotated by RoPE at each
+ * token's document position, rounded to bf16 (same page and section as
+ * llama_attn_quantize_e4m3; the QKV projection is one of the GEMMs it
+ * quantizes; RoPE as for llama_attn_prefill).
+ *
+ *   x    [B*S, d_model] E4M3 codes of the activations (row-major), s_x its scale
+ *   w    [N, d_model] E4M3 codes of the weight, N = (Hq + 2 Hkv) * D: rows
+ *        0 .. Hq*D-1 are the query heads, then Hkv key heads, then Hkv value
+ *        heads (the transpose of the page's K x N weight); s_w its scale
+ *   s_x, s_w  device floats (as written by llama_attn_quantize_e4m3)
+ *   q    [B, S, Hq, D] bf16 out, rotated; k [B, S, Hkv, D] bf16 out, rotated;
+ *   v    [B, S, Hkv, D] bf16 out
+ *   doc_offsets: as for llama_attn_prefill (positions restart per document)
+ * D == 128 and d_model % 128 == 0 (else LLAMA_ATTN_ERR_UNSUPPORTED); all
+ * tensors 16-byte aligned. Outputs must not alias inputs.
+ */
+int llama_attn_qkv_fp8_rope(const uint8_t *x, const float *s_x, const uint8_t *w, const float *s_w,
+                            llama_attn_bf16 *q, llama_attn_bf16 *k, llama_attn_bf16 *v,
+                            const int32_t *doc_offsets, int B, int S, int d_model, int Hq, int Hkv,
+                            int D, float rope_theta, cudaStream_t stream);
+
+/*
  * Prefill in true fp32 arithmetic on CUDA cores (FFMA, accurate expf), same
  * semantics and layouts as llama_attn_prefill with float tensors.
  * D even, 2 <= D <= 128.
