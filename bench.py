@@ -294,6 +294,7 @@ def run_ours(args, w):
     del hq, hk, hv, hout, dq, dk, dv, dout
 
     decode = None if args.no_decode else run_decode(args, la, dev, world, rank, hbm_peak, peak_kind)
+    qkv = run_qkv_fp8(args, la, dev, wr, tc_peak, peak_kind) if args.qkv_fp8 else None
     if la.llama_attn_get_device_error() != 0:
         raise RuntimeError("device error word set during the benchmark")
 
@@ -316,9 +317,11 @@ def run_ours(args, w):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clk,
-        "gpu_launches": launches + (decode["gpu_launches"] if decode else 0),
+        "gpu_launches": launches + (decode["gpu_launches"] if decode else 0) + (qkv["gpu_launches"] if qkv else 0),
         "decode": decode,
     }
+    if qkv is not None:
+        line["qkv_fp8"] = qkv
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -436,6 +439,59 @@ def run_cp(args, w):
         dist.destroy_process_group()
 
 
+def run_qkv_fp8(args, la, dev, w, tc_peak, peak_kind):
+    """The FP8 E4M3 QKV projection with RoPE for the prefill workload's tokens
+    (d_model = 128 * Hq, the Llama 3 width for these head counts): per step the
+    per-tensor quantization of X plus the projection GEMM with its RoPE
+    epilogue; the weight is quantized once, outside the timed region."""
+    d_model = 128 * w.Hq
+    M, N = w.B * w.S, (w.Hq + 2 * w.Hkv) * 128
+    g = torch.Generator(device=dev).manual_seed(w.seed + 17)
+    x = torch.randn(M, d_model, device=dev, generator=g).to(torch.bfloat16)
+    wt = (torch.randn(N, d_model, device=dev, generator=g) * d_model ** -0.5).to(torch.bfloat16)
+    inp_offs = W.make_prefill_inputs(w)["doc_offsets"]
+    offs = inp_offs.to(dev) if inp_offs is not None else None
+    wc, sw = la.llama_attn_quantize_e4m3(wt)
+    xc, sx = la.llama_attn_quantize_e4m3(x)
+    q = torch.empty(w.B, w.S, w.Hq, 128, dtype=torch.bfloat16, device=dev)
+    k = torch.empty(w.B, w.S, w.Hkv, 128, dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        la.llama_attn_quantize_e4m3(x, y=xc, scale=sx)
+        la.llama_attn_qkv_fp8_rope(xc, sx, wc, sw, w.B, w.S, w.Hq, w.Hkv, doc_offsets=offs,
+                                   rope_theta=w.rope_theta, q=q, k=k, v=v)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(args.steps, 10)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    la.llama_attn_profile_begin()
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    main_ms, main_n, launches = la.llama_attn_profile_end()
+    step_ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    flops = 2.0 * M * N * d_model
+    kernel_ms = main_ms / max(main_n, 1)
+    fp8_peak = 2.0 * tc_peak
+    return {
+        "workload": f"qkv_fp8_rope_M{M}_K{d_model}_N{N} ({w.name} tokens)", "value": flops / (step_ms / 1e3) / 1e12,
+        "unit": "TFLOP/s", "steps": steps, "ms_per_step": step_ms,
+        "roofline": {"bound": "tensor", "achieved": flops / (kernel_ms / 1e3) / 1e12, "peak": fp8_peak,
+                     "unit": "TFLOP/s", "frac": flops / (kernel_ms / 1e3) / 1e12 / fp8_peak,
+                     "peak_kind": f"2 x {peak_kind} bf16 dense burst (nominal fp8:bf16 ratio)",
+                     "kernel": "qkv_fp8_rope_kernel", "kernel_ms": kernel_ms, "traffic": None},
+        "gpu_launches": launches,
+    }
+
+
 def run_decode(args, la, dev, world, rank, hbm_peak, peak_kind):
     w = W.DECODE_70B
     nseq = args.decode_seqs
@@ -550,6 +606,8 @@ def main():
     ap.add_argument("--decode-page-size", type=int, default=0,
                     help="time the decode through the paged-cache entry point with this page size")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--qkv-fp8", action="store_true",
+                    help="also time the FP8 QKV projection with RoPE on the workload's tokens")
     ap.add_argument("--cp", action="store_true",
                     help="context-parallel prefill of the workload over the GPUs (strong scaling)")
     args = ap.parse_args()
