@@ -487,7 +487,8 @@ def run_qkv_fp8(args, la, dev, w, tc_peak, peak_kind):
         "roofline": {"bound": "tensor", "achieved": flops / (kernel_ms / 1e3) / 1e12, "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": flops / (kernel_ms / 1e3) / 1e12 / fp8_peak,
                      "peak_kind": f"2 x {peak_kind} bf16 dense burst (nominal fp8:bf16 ratio)",
-                     "kernel": "qkv_fp8_rope_kernel", "kernel_ms": kernel_ms, "traffic": None},
+                     "kernel": "qkv_fp8_rope_kernel", "kernel_ms": kernel_ms,
+                     "traffic": load_traffic("qkv_fp8_rope_kernel", f"qkv_fp8_rope_M{M}_K{d_model}_N{N}")},
         "gpu_launches": launches,
     }
 

@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       bool ok = true;
       auto load = [&](const CUtensorMap* tm, int g, int kv_row, int b) -> bool {
         const uint32_t st = idx % NSTAGE, use = idx / NSTAGE;
-        if (use > 0 && !mbar_wait(bar(B_KV_EMPTY + st), (use - 1) & 1, wc)) return false;
+        if (use > 0 && !mbar_wait_backoff(bar(B_KV_EMPTY + st), (use - 1) & 1, wc)) return false;
         mbar_arrive_expect_tx(bar(B_KV_FULL + st), TILE);
         tma_load_4d(sbase + OFF_KV + st * TILE, tm, bar(B_KV_FULL + st), 0, g, kv_row, b);
         tma_load_4d(sbase + OFF_KV + st * TILE + HALF, tm, bar(B_KV_FULL + st), 64, g, kv_row, b);
@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       publish(0, item < n_items ? item : -1);
       prefetch_rows(item);
       for (;; ++it) {
-        if (it > 0 && !mbar_wait(bar(B_Q_FREE), (it - 1) & 1, wc)) {
+        if (it > 0 && !mbar_wait_backoff(bar(B_Q_FREE), (it - 1) & 1, wc)) {
           ok = false;
           break;
         }
@@ -348,12 +348,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (lane == 0) {
       bool ok = true;
       for (int it = 0; ok; ++it) {
-        if (!mbar_wait(bar(B_O_STAGED + 0), it & 1, wc)) break;
+        if (!mbar_wait_backoff(bar(B_O_STAGED + 0), it & 1, wc)) break;
         const int item = ring_item[it % kItemRing];
         if (item < 0 || item >= n_items) break;
         const Item I = item_of(item, p);
         for (int s = 0; ok && s < p.NH; ++s) {
-          if (s > 0 && !mbar_wait(bar(B_O_STAGED + s), it & 1, wc)) {
+          if (s > 0 && !mbar_wait_backoff(bar(B_O_STAGED + s), it & 1, wc)) {
             ok = false;
             break;
           }

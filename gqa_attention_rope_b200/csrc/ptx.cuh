@@ -96,6 +96,36 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   }
 }
 
+// Bounded wait for waiters with slack (a producer several stages ahead, a
+// store warp): a non-blocking test with a short sleep between polls, so the
+// waiting warp leaves issue slots to the compute warps of its SM sub-partition.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_backoff(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(100);
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (w.aborted()) return false;
+      if (global_ns() - t0 > kWaitTimeoutNs) {
+        raise_error(LLAMA_ATTN_DEVERR_TIMEOUT);
+        atomicExch(&g_abort_epoch, w.epoch);
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- proxies
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
