@@ -475,8 +475,8 @@ int llama_attn_quantize_e4m3(const llama_attn_bf16* x, int64_t n, uint8_t* y, fl
   const int64_t nvec = n / 8;
   int n_sm = 148;
   if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
-  int64_t g = (nvec + 255) / 256;
-  const int grid = static_cast<int>(g < 4 * n_sm ? g : 4 * n_sm);
+  const int64_t g = (nvec + 1023) / 1024;  // four vectors per thread step
+  const int grid = static_cast<int>(g < 8 * n_sm ? g : 8 * n_sm);
   prof_count(2);
   la::q8::amax_bf16_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(x), nvec, dc.amax);
   LA_CUDA(cudaGetLastError());

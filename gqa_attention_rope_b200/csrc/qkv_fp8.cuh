@@ -25,12 +25,22 @@ constexpr float kE4M3Max = 448.f;
 // at launch.
 __global__ void amax_bf16_kernel(const uint4* __restrict__ x, int64_t n_vec, unsigned int* __restrict__ amax_bits) {
   float m = 0.f;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n_vec;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const uint4 v = x[i];
-    const float2 a = unpack_bf16x2(v.x), b = unpack_bf16x2(v.y), c = unpack_bf16x2(v.z), d = unpack_bf16x2(v.w);
-    m = fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(b.x), fabsf(b.y))));
-    m = fmaxf(m, fmaxf(fmaxf(fabsf(c.x), fabsf(c.y)), fmaxf(fabsf(d.x), fabsf(d.y))));
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  // four independent 16-byte loads in flight per thread
+  for (int64_t i0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i0 < n_vec; i0 += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * stride;
+      v[u] = i < n_vec ? x[i] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 a = unpack_bf16x2(v[u].x), b = unpack_bf16x2(v[u].y), c = unpack_bf16x2(v[u].z),
+                   d = unpack_bf16x2(v[u].w);
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(b.x), fabsf(b.y))));
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(c.x), fabsf(c.y)), fmaxf(fabsf(d.x), fabsf(d.y))));
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -59,15 +69,26 @@ __global__ void quantize_e4m3_kernel(const uint4* __restrict__ x, int64_t n_vec,
                                      float* __restrict__ scale_out) {
   const float s = scale_of(*amax_bits);
   if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n_vec;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const uint4 v = x[i];
-    const float2 a = unpack_bf16x2(v.x), b = unpack_bf16x2(v.y), c = unpack_bf16x2(v.z), d = unpack_bf16x2(v.w);
-    const uint32_t lo = e4m3x2(__fdiv_rn(a.x, s), __fdiv_rn(a.y, s)) |
-                        (e4m3x2(__fdiv_rn(b.x, s), __fdiv_rn(b.y, s)) << 16);
-    const uint32_t hi = e4m3x2(__fdiv_rn(c.x, s), __fdiv_rn(c.y, s)) |
-                        (e4m3x2(__fdiv_rn(d.x, s), __fdiv_rn(d.y, s)) << 16);
-    y[i] = make_uint2(lo, hi);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i0 = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i0 < n_vec; i0 += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * stride;
+      v[u] = i < n_vec ? x[i] : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i >= n_vec) break;
+      const float2 a = unpack_bf16x2(v[u].x), b = unpack_bf16x2(v[u].y), c = unpack_bf16x2(v[u].z),
+                   d = unpack_bf16x2(v[u].w);
+      const uint32_t lo = e4m3x2(__fdiv_rn(a.x, s), __fdiv_rn(a.y, s)) |
+                          (e4m3x2(__fdiv_rn(b.x, s), __fdiv_rn(b.y, s)) << 16);
+      const uint32_t hi = e4m3x2(__fdiv_rn(c.x, s), __fdiv_rn(c.y, s)) |
+                          (e4m3x2(__fdiv_rn(d.x, s), __fdiv_rn(d.y, s)) << 16);
+      y[i] = make_uint2(lo, hi);
+    }
   }
 }
 
