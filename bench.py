@@ -295,6 +295,7 @@ def run_ours(args, w):
 
     decode = None if args.no_decode else run_decode(args, la, dev, world, rank, hbm_peak, peak_kind)
     qkv = run_qkv_fp8(args, la, dev, wr, tc_peak, peak_kind) if args.qkv_fp8 else None
+    pex = run_prefill_ex(args, la, dev, wr, q, k, v, offs, flops, tc_peak, peak_kind) if args.prefill_ex else None
     if la.llama_attn_get_device_error() != 0:
         raise RuntimeError("device error word set during the benchmark")
 
@@ -317,11 +318,14 @@ def run_ours(args, w):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": clk,
-        "gpu_launches": launches + (decode["gpu_launches"] if decode else 0) + (qkv["gpu_launches"] if qkv else 0),
+        "gpu_launches": (launches + (decode["gpu_launches"] if decode else 0) + (qkv["gpu_launches"] if qkv else 0)
+                         + (pex["gpu_launches"] if pex else 0)),
         "decode": decode,
     }
     if qkv is not None:
         line["qkv_fp8"] = qkv
+    if pex is not None:
+        line["prefill_ex"] = pex
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -437,6 +441,46 @@ def run_cp(args, w):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_prefill_ex(args, la, dev, w, q, k, v, offs, flops, tc_peak, peak_kind):
+    """The prefill step with its two decode-linking outputs: per-row LSE and the
+    append of rotated K and V to a [B, Hkv, S, D] decode-layout cache."""
+    out = torch.empty_like(q)
+    lse = torch.empty(w.B, w.S, w.Hq, dtype=torch.float32, device=dev)
+    kc = torch.empty(w.B, w.Hkv, w.S, w.D, dtype=torch.bfloat16, device=dev)
+    vc = torch.empty_like(kc)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        la.llama_attn_prefill_ex(q, k, v, out=out, lse=lse, doc_offsets=offs, rope_theta=w.rope_theta,
+                                 kcache=kc, vcache=vc)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(args.steps, 10)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    la.llama_attn_profile_begin()
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    main_ms, main_n, launches = la.llama_attn_profile_end()
+    step_ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    kernel_ms = main_ms / max(main_n, 1)
+    return {
+        "workload": w.name + " + lse + kv cache append", "value": flops / (step_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+        "steps": steps, "ms_per_step": step_ms,
+        "roofline": {"bound": "tensor", "achieved": flops / (kernel_ms / 1e3) / 1e12, "peak": tc_peak,
+                     "unit": "TFLOP/s", "frac": flops / (kernel_ms / 1e3) / 1e12 / tc_peak,
+                     "peak_kind": f"{peak_kind} bf16 dense (burst)", "kernel": "prefill_bf16_kernel",
+                     "kernel_ms": kernel_ms, "traffic": None},
+        "gpu_launches": launches,
+    }
 
 
 def run_qkv_fp8(args, la, dev, w, tc_peak, peak_kind):
@@ -607,6 +651,8 @@ def main():
     ap.add_argument("--decode-page-size", type=int, default=0,
                     help="time the decode through the paged-cache entry point with this page size")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--prefill-ex", action="store_true",
+                    help="also time the prefill with LSE output and KV-cache append")
     ap.add_argument("--qkv-fp8", action="store_true",
                     help="also time the FP8 QKV projection with RoPE on the workload's tokens")
     ap.add_argument("--cp", action="store_true",
