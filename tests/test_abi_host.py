@@ -98,6 +98,39 @@ def test_decode_rejects(lib):
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 16, 2, 128, 64, 5e5, ctypes.c_void_p(4100), big, None) == WORKSPACE
 
 
+@pytest.mark.parametrize("args,expect", [
+    # q, k, v, out, lse, B, Sq, Skv, Hq, Hkv, D, q_pos_a, q_split, q_pos_b, theta
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 256, 1024, 8, 2, 128, 64, 128, 512, 5e5), INVALID),   # position not /128
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 256, 1024, 8, 2, 128, 0, 100, 512, 5e5), INVALID),    # split not /128
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 256, 1024, 8, 2, 128, 0, 384, 0, 5e5), INVALID),      # split > Sq
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 256, 1024, 8, 2, 128, 0, 128, 1000, 5e5), INVALID),   # chunk b past Skv
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 256, 1024, 8, 2, 128, 1024, 128, 0, 5e5), INVALID),   # chunk a past Skv
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 256, 0, 8, 2, 128, 0, 128, 0, 5e5), INVALID),         # Skv = 0
+    ((None, FAKE, FAKE, FAKE, None, 1, 256, 1024, 8, 2, 128, 0, 128, 512, 5e5), INVALID),
+    ((FAKE, FAKE, FAKE, FAKE, None, 1, 256, 1024, 8, 2, 64, 0, 128, 512, 5e5), UNSUPPORTED),
+])
+def test_prefill_cp_rejects(lib, args, expect):
+    assert lib.llama_attn_prefill_cp(*args, None) == expect
+
+
+def test_fp8_entries_reject(lib):
+    q = lib.llama_attn_quantize_e4m3
+    assert q(None, 64, FAKE, FAKE, None) == INVALID
+    assert q(FAKE, 12, FAKE, FAKE, None) == INVALID              # n % 8 != 0
+    assert q(FAKE, 0, FAKE, FAKE, None) == INVALID
+    assert q(ctypes.c_void_p(4104), 64, FAKE, FAKE, None) == INVALID  # x not 16-byte aligned
+    g = lib.llama_attn_qkv_fp8_rope
+    # x, s_x, w, s_w, q, k, v, offs, B, S, d_model, Hq, Hkv, D, theta
+    assert g(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 128, 256, 4, 2, 128, 5e5, None) == INVALID
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 128, 200, 4, 2, 128, 5e5, None) == UNSUPPORTED
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 128, 256, 4, 2, 64, 5e5, None) == UNSUPPORTED
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, 128, 256, 4, 2, 128, 5e5, None) == INVALID
+    assert g(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 128, 256, 4, 2, 128, 0.0, None) == INVALID
+    r = lib.llama_attn_prefill_rotated
+    assert r(None, FAKE, FAKE, FAKE, None, None, 1, 128, 8, 2, 128, None) == INVALID
+    assert r(FAKE, FAKE, FAKE, FAKE, None, None, 1, 128, 8, 2, 64, None) == UNSUPPORTED
+
+
 def test_python_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(RuntimeError, match="not found"):
         la.load_library(str(tmp_path / "missing.so"))
