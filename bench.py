@@ -15,6 +15,13 @@ a bounded sample of query rows of the same workload, in the same unit.
 Multi-GPU (torchrun): one process per GPU, each with its own independent
 batch (weak scaling, no data-path collective); rank 0 prints the line, value =
 FLOPs of all ranks / max-over-ranks time.
+
+Options that add measurements of the paths around the hot path:
+  --cp               context-parallel prefill of one single-document workload
+                     over the GPUs (zigzag split, K/V all-gather, strong scaling)
+  --prefill-ex       the prefill with its LSE output and KV-cache append
+  --decode-page-size the decode through the paged-cache entry point
+  --qkv-fp8          the FP8 E4M3 QKV projection with RoPE on the workload's tokens
 """
 from __future__ import annotations
 
