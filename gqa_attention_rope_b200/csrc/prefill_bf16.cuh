@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(bar(B_KV_EMPTY + s), 1);
     }
     mbar_init(bar(B_Q_FULL), 1);
-    mbar_init(bar(B_Q_FREE), 1);
+    mbar_init(bar(B_Q_FREE), 2);  // the S issuer's commit and the PV issuer's arrival
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(B_Q_READY + s), 128);
       mbar_init(bar(B_S_READY + s), 1);
@@ -275,6 +275,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       uint32_t ring = 0, tiles = 0;
       for (int it = 0; ok; ++it) {
         if (!mbar_wait(bar(B_Q_FULL), it & 1, wc)) break;
+        // The PV issuer waits on Q_FULL only to learn the item id; its arrival
+        // on Q_FREE keeps the next Q load behind this wait, so its parity wait
+        // can never fall two phases behind.
+        if (warp == 2) mbar_arrive(bar(B_Q_FREE));
         const int item = ring_item[it % kItemRing];
         if (item < 0 || item >= n_items) break;
         const Item I = item_of(item, p);
