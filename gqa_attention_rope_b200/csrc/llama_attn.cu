@@ -16,7 +16,7 @@
 #include "qkv_fp8.cuh"
 #include "decode.cuh"
 
-#define LLAMA_ATTN_VERSION 100  // 0.1.0
+#define LLAMA_ATTN_VERSION 200  // 0.2.0: context-parallel, pre-rotated and FP8 projection entry points
 
 namespace {
 

@@ -306,10 +306,10 @@ int llama_attn_get_device_error(cudaStream_t stream);
 
 /*
  * Benchmark instrumentation (host side, current device only).
- * llama_attn_profile_begin() starts a session: each later prefill / decode call
- * records a CUDA event pair on its stream around its main kernel (prefill: the
- * attention kernel; decode: the split-KV kernel) and every kernel the library
- * launches is counted. llama_attn_profile_end() waits for the recorded events,
+ * llama_attn_profile_begin() starts a session: each later prefill, decode or
+ * QKV projection call records a CUDA event pair on its stream around its main
+ * kernel (prefill: the attention kernel; decode: the split-KV kernel;
+ * projection: the FP8 GEMM) and every kernel the library launches is counted. llama_attn_profile_end() waits for the recorded events,
  * writes the summed main-kernel time in milliseconds, the number of timed main
  * kernels and the number of kernels launched, and ends the session. At most
  * 4096 main kernels are timed per session; later ones are counted only.
