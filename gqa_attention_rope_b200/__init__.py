@@ -342,6 +342,34 @@ def llama_attn_decode(q, kcache, vcache, cache_lens, out=None, workspace=None, r
     return out
 
 
+def llama_attn_decode_paged(q, kpages, vpages, block_table, cache_lens, out=None, workspace=None,
+                            rope_theta: float = 500000.0, stream=None):
+    """bf16 decode against a paged cache. q [B,Hq,D]; kpages/vpages
+    [n_pages,Hkv,page_size,D] (keys pre-rotated); block_table int32 [B,max_blocks]
+    (logical block j of sequence b is page block_table[b, j]); cache_lens int32 [B]."""
+    import torch
+    _require(q.dim() == 3 and kpages.dim() == 4 and vpages.shape == kpages.shape, "bad shapes")
+    for t in (q, kpages, vpages):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "bf16 contiguous CUDA tensors expected")
+    for t in (block_table, cache_lens):
+        _require(t.is_cuda and t.dtype == torch.int32 and t.is_contiguous(), "block_table / cache_lens: int32 CUDA")
+    B, Hq, D = q.shape
+    n_pages, Hkv, page_size = kpages.shape[0], kpages.shape[1], kpages.shape[2]
+    _require(kpages.shape[3] == D and block_table.dim() == 2 and block_table.shape[0] == B
+             and cache_lens.numel() == B, "bad shapes")
+    max_blocks = block_table.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    need = llama_attn_decode_workspace_size(B, Hq, max_blocks * page_size, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib().llama_attn_decode_paged(_ptr(q), _ptr(kpages), _ptr(vpages), _ptr(block_table), _ptr(cache_lens),
+                                       _ptr(out), B, Hq, Hkv, D, page_size, max_blocks, n_pages, float(rope_theta),
+                                       _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("llama_attn_decode_paged", st)
+    return out
+
+
 def llama_attn_decode_noalloc(q, kcache, vcache, cache_lens, out, rope_theta: float = 500000.0, stream=None):
     """llama_attn_decode without a workspace or any device allocation, for
     callers that cannot allocate: the partials go to a fixed 72 MiB array in the

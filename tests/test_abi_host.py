@@ -131,6 +131,11 @@ def test_fp8_entries_reject(lib):
     assert r(FAKE, FAKE, FAKE, FAKE, None, None, 1, 128, 8, 2, 64, None) == UNSUPPORTED
 
 
+def test_binding_wraps_every_exported_name():
+    for n in la.EXPORTED:
+        assert callable(getattr(la, n, None)), f"no Python wrapper named {n}"
+
+
 def test_python_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(RuntimeError, match="not found"):
         la.load_library(str(tmp_path / "missing.so"))

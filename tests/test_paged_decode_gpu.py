@@ -71,9 +71,12 @@ def test_paged_decode(page_size, lens):
                                      page_size, max_blocks, n_pages, ctypes.c_float(w.rope_theta), _p(ws), ws_bytes,
                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0
+    # the Python binding's wrapper makes the same call
+    out_py = la.llama_attn_decode_paged(q, kp, vp, table, lens_d, rope_theta=w.rope_theta)
     ref_gpu = la.llama_attn_decode(q, inp["kcache"].cuda(), inp["vcache"].cuda(), lens_d)
     torch.cuda.synchronize()
     assert torch.equal(out, ref_gpu), "paged decode differs from contiguous decode"
+    assert torch.equal(out_py, out), "binding wrapper differs from the direct call"
     ref = O.decode(inp["q"], inp["kcache"], inp["vcache"], inp["cache_lens"], w.rope_theta)
     err = np.abs(out.float().cpu().numpy() - ref).max()
     assert err <= TOL_BF16, f"max abs err {err}"
