@@ -36,6 +36,7 @@ MUTANTS = {
     "doc_position_not_restarted_inside_row": ("pos[t] = (int32_t)(t - start);",
                                               "pos[t] = (int32_t)(t - start + (t - start) / 2);"),
     "lse_drops_max": ("if (lse) *lse = m + log(sum);", "if (lse) *lse = log(sum);"),
+    "lse_base_two": ("if (lse) *lse = m + log(sum);", "if (lse) *lse = m + log2(sum);"),
 }
 
 

@@ -168,8 +168,20 @@ def pin_projection_rope(F):
     assert np.array_equal(vr.reshape(T, Hkv, D), v)
 
 
+GOLDEN = os.path.join(ROOT, "tests", "golden", "e4m3_rounding_examples.txt")
+
+
+def pin_golden_examples(F):
+    """Hand-worked values from the format definition (tests/golden)."""
+    rows = [ln.split() for ln in open(GOLDEN) if ln.strip() and not ln.startswith("#")]
+    for r in rows:
+        value, code = float(r[0]), int(r[1], 16)
+        got = int(F.e4m3_round(np.array([value]))[0])
+        assert got == code, f"{value}: code {got:#04x}, expected {code:#04x}"
+
+
 PINS = [pin_table, pin_round_brute, pin_round_torch, pin_roundtrip, pin_scaling, pin_projection_integer,
-        pin_projection_head_order, pin_projection_rope]
+        pin_projection_head_order, pin_projection_rope, pin_golden_examples]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=[p.__name__ for p in PINS])
