@@ -58,9 +58,14 @@ constexpr int NTHREADS = 384;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleLog2 = 8.0f;
 
+// Each ring stage has one full barrier per tile kind: a K tile landing in a
+// stage completes a phase of that stage's K_FULL barrier, a V tile one of its
+// V_FULL barrier. Each issuer waits only on its own kind, in consecutive
+// phases, so no wait depends on the order in which separate TMA loads land.
 enum : int {
-  B_KV_FULL = 0,
-  B_KV_EMPTY = B_KV_FULL + NSTAGE,
+  B_K_FULL = 0,
+  B_V_FULL = B_K_FULL + NSTAGE,
+  B_KV_EMPTY = B_V_FULL + NSTAGE,
   B_Q_FULL = B_KV_EMPTY + NSTAGE,
   B_Q_READY,
   B_S_READY = B_Q_READY + 2,
@@ -159,7 +164,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(bar(B_KV_FULL + s), 1);
+      mbar_init(bar(B_K_FULL + s), 1);
+      mbar_init(bar(B_V_FULL + s), 1);
       mbar_init(bar(B_KV_EMPTY + s), 1);
     }
     mbar_init(bar(B_Q_FULL), 1);
@@ -198,13 +204,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t idx = 0;  // running ring index
+      // Per stage and tile kind: bit st of *_any says a load of that kind went
+      // into stage st, bit st of *_par is the parity of their count.
+      uint32_t k_any = 0, k_par = 0, v_any = 0, v_par = 0;
       bool ok = true;
-      auto load = [&](const CUtensorMap* tm, int g, int kv_row, int b) -> bool {
+      auto load = [&](bool is_v, int g, int kv_row, int b) -> bool {
         const uint32_t st = idx % NSTAGE, use = idx / NSTAGE;
         if (use > 0 && !mbar_wait_backoff(bar(B_KV_EMPTY + st), (use - 1) & 1, wc)) return false;
-        mbar_arrive_expect_tx(bar(B_KV_FULL + st), TILE);
-        tma_load_4d(sbase + OFF_KV + st * TILE, tm, bar(B_KV_FULL + st), 0, g, kv_row, b);
-        tma_load_4d(sbase + OFF_KV + st * TILE + HALF, tm, bar(B_KV_FULL + st), 64, g, kv_row, b);
+        const uint32_t full = bar((is_v ? B_V_FULL : B_K_FULL) + static_cast<int>(st));
+        const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
+        mbar_arrive_expect_tx(full, TILE);
+        tma_load_4d(sbase + OFF_KV + st * TILE, tm, full, 0, g, kv_row, b);
+        tma_load_4d(sbase + OFF_KV + st * TILE + HALF, tm, full, 64, g, kv_row, b);
+        if (is_v) {
+          v_any |= 1u << st;
+          v_par ^= 1u << st;
+        } else {
+          k_any |= 1u << st;
+          k_par ^= 1u << st;
+        }
         ++idx;
         return true;
       };
@@ -248,10 +266,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         next_item = (item < n_items) ? atomicAdd(p.sched, 1) + static_cast<int>(gridDim.x) : n_items;
         publish(it + 1, item < n_items ? item : -1);
         prefetch_rows(item);
-        ok = load(&tm_k, I.g, I.kv_t0 * BN, I.b);
+        ok = load(false, I.g, I.kv_t0 * BN, I.b);
         for (int j = 1; ok && j < I.n_kv; ++j)
-          ok = load(&tm_k, I.g, (I.kv_t0 + j) * BN, I.b) && load(&tm_v, I.g, (I.kv_t0 + j - 1) * BN, I.b);
-        if (ok) ok = load(&tm_v, I.g, (I.kv_t0 + I.n_kv - 1) * BN, I.b);
+          ok = load(false, I.g, (I.kv_t0 + j) * BN, I.b) && load(true, I.g, (I.kv_t0 + j - 1) * BN, I.b);
+        if (ok) ok = load(true, I.g, (I.kv_t0 + I.n_kv - 1) * BN, I.b);
         if (!ok) {
           ++it;
           break;
@@ -260,8 +278,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // Every issued load has landed before this CTA may exit (these return at
       // once in the normal flow, where every load was consumed).
       if (!ended && it > 0) mbar_wait(bar(B_Q_FULL), (it - 1) & 1, wc);
-      for (uint32_t st = 0; st < NSTAGE; ++st)
-        if (idx > st) mbar_wait(bar(B_KV_FULL + st), ((idx - 1 - st) / NSTAGE) & 1, wc);
+      // Only the last load into a stage can still be in flight (each load
+      // waited for the stage to be emptied), so the latest phase of each
+      // kind's full barrier covers every load.
+      for (int st = 0; st < NSTAGE; ++st) {
+        if ((k_any >> st) & 1u) mbar_wait(bar(B_K_FULL + st), ((k_par >> st) & 1u) ^ 1u, wc);
+        if ((v_any >> st) & 1u) mbar_wait(bar(B_V_FULL + st), ((v_par >> st) & 1u) ^ 1u, wc);
+      }
     }
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------ MMA issuers
@@ -273,6 +296,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 128, 1);
       bool ok = true;
       uint32_t ring = 0, tiles = 0;
+      // bit st: parity of the next phase this issuer waits for on stage st's
+      // full barrier of its tile kind (K for the S issuer, V for the PV issuer)
+      uint32_t full_par = 0;
       for (int it = 0; ok; ++it) {
         if (!mbar_wait(bar(B_Q_FULL), it & 1, wc)) break;
         // The PV issuer waits on Q_FULL only to learn the item id; its arrival
@@ -288,10 +314,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const uint32_t idx = ring + ((j == 0) ? 0u : static_cast<uint32_t>(2 * j - 1));
             const uint32_t st = idx % NSTAGE;
             const uint32_t T = tiles + j;
-            if (!mbar_wait(bar(B_KV_FULL + st), (idx / NSTAGE) & 1, wc)) {
+            if (!mbar_wait(bar(B_K_FULL + static_cast<int>(st)), (full_par >> st) & 1u, wc)) {
               ok = false;
               break;
             }
+            full_par ^= 1u << st;
             const uint64_t db = kdesc(sbase + OFF_KV + st * TILE);
             for (int s = 0; s < p.NH; ++s) {
               if (T > 0 && !mbar_wait(bar(B_S_FREE + s), (T - 1) & 1, wc)) {
@@ -316,10 +343,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 ring + ((j < I.n_kv - 1) ? static_cast<uint32_t>(2 * j + 2) : static_cast<uint32_t>(2 * I.n_kv - 1));
             const uint32_t st = idx % NSTAGE;
             const uint32_t T = tiles + j;
-            if (!mbar_wait(bar(B_KV_FULL + st), (idx / NSTAGE) & 1, wc)) {
+            if (!mbar_wait(bar(B_V_FULL + static_cast<int>(st)), (full_par >> st) & 1u, wc)) {
               ok = false;
               break;
             }
+            full_par ^= 1u << st;
             const uint64_t db = vdesc(sbase + OFF_KV + st * TILE);
             for (int s = 0; s < p.NH; ++s) {
               if (!mbar_wait(bar(B_P_READY + s), T & 1, wc)) {
