@@ -33,6 +33,11 @@ EXPORTED = (
     "llama_attn_prefill_rotated",
     "llama_attn_quantize_e4m3",
     "llama_attn_qkv_fp8_rope",
+    "llama_attn_rope_table_size",
+    "llama_attn_rope_table_build",
+    "llama_attn_prefill_workspace_size",
+    "llama_attn_prefill_ws",
+    "llama_attn_prefill_cp_ws",
 )
 
 DEVERR_TIMEOUT = 0x1
@@ -90,6 +95,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.llama_attn_quantize_e4m3.restype = I
     lib.llama_attn_qkv_fp8_rope.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.llama_attn_qkv_fp8_rope.restype = I
+    lib.llama_attn_rope_table_size.argtypes = [I, I]
+    lib.llama_attn_rope_table_size.restype = Z
+    lib.llama_attn_rope_table_build.argtypes = [P, Z, I, I, F, P]
+    lib.llama_attn_rope_table_build.restype = I
+    lib.llama_attn_prefill_workspace_size.argtypes = [I, I, I, I]
+    lib.llama_attn_prefill_workspace_size.restype = Z
+    lib.llama_attn_prefill_ws.argtypes = [P, P, P, P, P, P, I, I, I, I, I, P, I, P, P, I, P, Z, P]
+    lib.llama_attn_prefill_ws.restype = I
+    lib.llama_attn_prefill_cp_ws.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, I, P, Z, P]
+    lib.llama_attn_prefill_cp_ws.restype = I
     return lib
 
 
@@ -224,6 +239,95 @@ def llama_attn_prefill_cp(q, k, v, q_pos_a: int, q_split: int, q_pos_b: int = 0,
     st = lib().llama_attn_prefill_cp(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Skv, Hq, Hkv, D,
                                      int(q_pos_a), int(q_split), int(q_pos_b), float(rope_theta), _stream(stream))
     _check("llama_attn_prefill_cp", st)
+    return out, lse
+
+
+def llama_attn_rope_table_size(maxpos: int, D: int = 128) -> int:
+    return int(lib().llama_attn_rope_table_size(int(maxpos), int(D)))
+
+
+def llama_attn_rope_table_build(maxpos: int, D: int = 128, rope_theta: float = 500000.0, table=None, device=None,
+                                stream=None):
+    """Caller-owned RoPE table for the *_ws entry points: float32 [maxpos, D/2, 2]
+    holding (cos, sin) of p * theta_k. Allocated here unless ``table`` is given."""
+    import torch
+    need = llama_attn_rope_table_size(maxpos, D)
+    _require(need > 0, "maxpos >= 1 and even D in [2, 128]")
+    if table is None:
+        table = torch.empty(maxpos, D // 2, 2, dtype=torch.float32,
+                            device=device if device is not None else torch.cuda.current_device())
+    _require(table.is_cuda and table.is_contiguous(), "table: contiguous CUDA tensor")
+    st = lib().llama_attn_rope_table_build(_ptr(table), table.numel() * table.element_size(), int(maxpos), int(D),
+                                           float(rope_theta), _stream(stream))
+    _check("llama_attn_rope_table_build", st)
+    return table
+
+
+def llama_attn_prefill_workspace_size(B: int, S: int, Hkv: int, D: int = 128) -> int:
+    return int(lib().llama_attn_prefill_workspace_size(int(B), int(S), int(Hkv), int(D)))
+
+
+def _table_rows(table):
+    return table.shape[0] if table.dim() >= 1 else 0
+
+
+def llama_attn_prefill_ws(q, k, v, rope_table, workspace, out=None, lse=None, doc_offsets=None, kcache=None,
+                          vcache=None, stream=None):
+    """llama_attn_prefill_ex with caller-owned memory: ``rope_table`` from
+    llama_attn_rope_table_build (rows >= S) and ``workspace`` a CUDA buffer of at
+    least llama_attn_prefill_workspace_size(B, S, Hkv) bytes. The call allocates
+    nothing and does not synchronise (``out`` is allocated here only when not
+    given). Returns (out, lse)."""
+    import torch
+    _require(q.dim() == 4 and k.dim() == 4 and v.dim() == 4, "q, k, v must be [B, S, H, D]")
+    for t in (q, k, v):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "bf16 contiguous CUDA tensors expected")
+    B, S, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _require(k.shape == (B, S, Hkv, D) and v.shape == k.shape, "k and v must be [B, S, Hkv, D]")
+    if out is None:
+        out = torch.empty_like(q)
+    _require(out.shape == q.shape and out.dtype == torch.bfloat16 and out.is_contiguous(), "bad out")
+    if lse is not None:
+        _require(lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.shape == (B, S, Hq),
+                 "lse: float32 [B, S, Hq]")
+    Lmax = 0
+    if kcache is not None or vcache is not None:
+        _require(kcache is not None and vcache is not None and kcache.shape == vcache.shape, "kcache and vcache")
+        _require(kcache.shape[0] == B and kcache.shape[1] == Hkv and kcache.shape[3] == D, "cache shape")
+        Lmax = kcache.shape[2]
+    if doc_offsets is not None:
+        _require(doc_offsets.is_cuda and doc_offsets.dtype == torch.int32, "doc_offsets: int32 CUDA tensor")
+    _require(rope_table.is_cuda and workspace.is_cuda, "rope_table and workspace: CUDA tensors")
+    st = lib().llama_attn_prefill_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(doc_offsets), B, S, Hq,
+                                     Hkv, D, _ptr(rope_table), _table_rows(rope_table), _ptr(kcache), _ptr(vcache),
+                                     Lmax, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                     _stream(stream))
+    _check("llama_attn_prefill_ws", st)
+    return out, lse
+
+
+def llama_attn_prefill_cp_ws(q, k, v, q_pos_a: int, q_split: int, q_pos_b: int, rope_table, workspace, out=None,
+                             lse=None, stream=None):
+    """llama_attn_prefill_cp with caller-owned memory (rope_table rows >= Skv,
+    workspace of llama_attn_prefill_workspace_size(B, Skv, Hkv) bytes). Returns (out, lse)."""
+    import torch
+    _require(q.dim() == 4 and k.dim() == 4 and v.dim() == 4, "q, k, v must be [B, S, H, D]")
+    for t in (q, k, v):
+        _require(t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous(), "bf16 contiguous CUDA tensors expected")
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    _require(k.shape == (B, Skv, Hkv, D) and v.shape == k.shape, "k and v must be [B, Skv, Hkv, D]")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is not None:
+        _require(lse.is_cuda and lse.dtype == torch.float32 and lse.is_contiguous() and lse.shape == (B, Sq, Hq),
+                 "lse: float32 [B, Sq, Hq]")
+    st = lib().llama_attn_prefill_cp_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Sq, Skv, Hq, Hkv, D,
+                                        int(q_pos_a), int(q_split), int(q_pos_b), _ptr(rope_table),
+                                        _table_rows(rope_table), _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("llama_attn_prefill_cp_ws", st)
     return out, lse
 
 

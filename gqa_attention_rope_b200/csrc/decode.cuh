@@ -34,22 +34,20 @@ constexpr int NTHREADS = (NCW + 1) * 32;
 constexpr uint32_t KHALF = ROWS * 128;      // 64 rows x 64 bf16 = 8 KB
 constexpr uint32_t STAGE = 4 * KHALF;       // K (2 halves) + V (2 halves)
 constexpr uint32_t OFF_BAR = NSTAGE * STAGE;
-constexpr uint32_t SMEM_ALLOC = OFF_BAR + 64 + 1024;
-// The variant that computes its own (cos, sin) row keeps it after the barriers.
-constexpr uint32_t OFF_SELF_TABLE = OFF_BAR + 64;
-constexpr uint32_t SMEM_ALLOC_SELF_TABLE = SMEM_ALLOC + 64 * 8;
+// The CTA's (cos, sin) row at position len sits after the barriers.
+constexpr uint32_t OFF_ROPE_ROW = OFF_BAR + 64;
+constexpr uint32_t SMEM_ALLOC = OFF_ROPE_ROW + 64 * 8 + 1024;
 static_assert(NCW * (2 * 16 + 16 * 128) * 4 <= OFF_BAR, "combine scratch fits in the ring");
 
 struct Params {
   int B, Hq, Hkv, G, Lmax, nchunk;
   const int32_t* lens;
   const uint16_t* q;         // [B, Hq, 128] bf16 bits
-  const float4* rope_tab;    // (cos, sin) pairs, 64 per position
   float scale_log2;
   float* part_o;             // [B, Hq, nchunk, 128]
   float* part_lse;           // [B, Hq, nchunk]
   unsigned int epoch;        // launch id for bounded-wait abort propagation
-  double rope_theta;         // used only when the kernel forms its own (cos, sin) row
+  double rope_theta;         // RoPE base; the CTA forms the (cos, sin) row of position len itself
   // paged cache (kPaged): logical row n of sequence b lives in page
   // block_table[b * max_blocks + n / page_size] at row n % page_size; the page
   // pool is [n_pages, Hkv, page_size, 128], page_size a multiple of ROWS.
@@ -59,11 +57,11 @@ struct Params {
 
 __device__ __forceinline__ int valid_len(int len, int Lmax) { return (len < 0 || len > Lmax) ? 0 : len; }
 
-// kSelfTable = false: (cos, sin) at position len come from the cached table
-// p.rope_tab. kSelfTable = true: the CTA forms that one row itself (float64
-// angle, same formula as rope_table_kernel) in shared memory, so no table needs
-// to be allocated.
-template <bool kSelfTable, bool kPaged = false>
+// The query is rotated at position len: the CTA forms that one (cos, sin) row
+// itself (float64 angle, the formula of rope_table_kernel) in shared memory,
+// so the decode needs no table. The compute warps build it after the block
+// barrier, so the producer's first loads are not held back by it.
+template <bool kPaged = false>
 __global__ void __launch_bounds__(NTHREADS, 2)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const Params p) {
@@ -92,15 +90,6 @@ __global__ void __launch_bounds__(NTHREADS, 2)
     fence_mbar_init();
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
-  }
-  if constexpr (kSelfTable) {
-    if (threadIdx.x < 64) {
-      const double freq = pow(p.rope_theta, -2.0 * static_cast<double>(threadIdx.x) / 128.0);
-      double sn, cs;
-      sincos(static_cast<double>(len) * freq, &sn, &cs);
-      reinterpret_cast<float2*>(smem + OFF_SELF_TABLE)[threadIdx.x] =
-          make_float2(static_cast<float>(cs), static_cast<float>(sn));
-    }
   }
   __syncthreads();
 
@@ -140,10 +129,17 @@ __global__ void __launch_bounds__(NTHREADS, 2)
   const int gq = lane >> 2, t = lane & 3;  // fragment row group / thread-in-group
   const int G = p.G;
   // A fragments of the rotated query: rows = heads of the group (row >= G is zero).
+  if (threadIdx.x < 64) {
+    const double freq = pow(p.rope_theta, -2.0 * static_cast<double>(threadIdx.x) / 128.0);
+    double sn, cs;
+    sincos(static_cast<double>(len) * freq, &sn, &cs);
+    reinterpret_cast<float2*>(smem + OFF_ROPE_ROW)[threadIdx.x] =
+        make_float2(static_cast<float>(cs), static_cast<float>(sn));
+  }
+  asm volatile("bar.sync 2, %0;" ::"r"(NCW * 32) : "memory");  // the compute warps only
   uint32_t qa[8][4];
   {
-    const float4* tab = kSelfTable ? reinterpret_cast<const float4*>(smem + OFF_SELF_TABLE)
-                                   : p.rope_tab + static_cast<int64_t>(len) * 32;
+    const float4* tab = reinterpret_cast<const float4*>(smem + OFF_ROPE_ROW);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
 #pragma unroll
@@ -154,7 +150,7 @@ __global__ void __launch_bounds__(NTHREADS, 2)
         if (row < G) {
           const uint32_t x = *reinterpret_cast<const uint32_t*>(
               p.q + (static_cast<int64_t>(b) * p.Hq + gk * G + row) * 128 + d);
-          const float4 cs = kSelfTable ? tab[d >> 2] : __ldg(tab + (d >> 2));
+          const float4 cs = tab[d >> 2];
           const float cc = (d & 2) ? cs.z : cs.x, ss = (d & 2) ? cs.w : cs.y;
           val = rope_rotate_pair(x, cc, ss);
         }

@@ -3,6 +3,7 @@
 // kernel launches behind the C ABI declared in include/llama_attn.h.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -16,7 +17,7 @@
 #include "qkv_fp8.cuh"
 #include "decode.cuh"
 
-#define LLAMA_ATTN_VERSION 200  // 0.2.0: context-parallel, pre-rotated and FP8 projection entry points
+#define LLAMA_ATTN_VERSION 300  // 0.3.0: caller-workspace prefill entry points, caller-owned RoPE table
 
 namespace {
 
@@ -29,28 +30,34 @@ struct RopeTable {
   float2* ptr = nullptr;
 };
 
+// Library-owned buffers behind the convenience entry points (the *_ws entry
+// points take caller memory instead and touch none of these).
 struct DeviceCache {
   std::vector<RopeTable> tables;
-  void* krot = nullptr;
-  size_t krot_bytes = 0;
-  int32_t* doc_start = nullptr;
-  size_t doc_bytes = 0;
-  int* sched = nullptr;  // work-item counter of the persistent prefill kernel
-  bool prefill_attr_set = false;
-  bool decode_attr_set = false;
-  bool decode_paged_attr_set = false;
+  void* prefill_ws = nullptr;  // rotated K, document starts, work-item counter
+  size_t prefill_ws_bytes = 0;
   unsigned int* amax = nullptr;  // per-tensor amax of the E4M3 quantizer
-  bool qkv_attr_set = false;
+  int32_t* doc_start = nullptr;  // document starts of the fp32 and FP8 paths
+  size_t doc_bytes = 0;
+};
+
+// Per-device launch settings, set once (kernel attributes, SM count).
+struct DeviceSetup {
+  std::once_flag once;
+  int status = 0;
+  int n_sm = 148;
 };
 
 std::mutex g_mutex;
 DeviceCache g_cache[kMaxDevices];
-unsigned int g_epoch = 0;
+DeviceSetup g_setup[kMaxDevices];
+std::atomic<unsigned int> g_epoch{0};
 
 // Distinct, nonzero id per launch that uses bounded waits.
 unsigned int next_epoch() {
-  if (++g_epoch == 0) ++g_epoch;
-  return g_epoch;
+  unsigned int e = ++g_epoch;
+  if (e == 0) e = ++g_epoch;
+  return e;
 }
 
 // ---- benchmark instrumentation (see llama_attn_profile_begin)
@@ -235,6 +242,29 @@ int check_prefill_common(const void* q, const void* k, const void* v, const void
   return LLAMA_ATTN_OK;
 }
 
+// Once per device: the kernels' shared-memory attributes and the SM count.
+// Thread-safe; no allocation, no synchronisation.
+int device_setup(int dev, int* n_sm) {
+  DeviceSetup& ds = g_setup[dev];
+  std::call_once(ds.once, [&] {
+    int st = LLAMA_ATTN_OK;
+    auto attr = [&](const void* fn, uint32_t bytes) {
+      if (st == LLAMA_ATTN_OK &&
+          cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) != cudaSuccess)
+        st = LLAMA_ATTN_ERR_CUDA;
+    };
+    attr(reinterpret_cast<const void*>(la::pfx::prefill_bf16_kernel), la::pfx::SMEM_ALLOC);
+    attr(reinterpret_cast<const void*>(la::dec::decode_split_kernel<false>), la::dec::SMEM_ALLOC);
+    attr(reinterpret_cast<const void*>(la::dec::decode_split_kernel<true>), la::dec::SMEM_ALLOC);
+    attr(reinterpret_cast<const void*>(la::q8::qkv_fp8_rope_kernel), la::q8::SMEM_ALLOC);
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0) ds.n_sm = n;
+    ds.status = st;
+  });
+  if (n_sm) *n_sm = ds.n_sm;
+  return ds.status;
+}
+
 }  // namespace
 
 // ---- scratch for llama_attn_decode_noalloc
@@ -247,7 +277,6 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 namespace {
 void* g_noalloc_scratch_addr[kMaxDevices];
-bool g_noalloc_attr_set[kMaxDevices];
 }  // namespace
 
 extern "C" {
@@ -291,7 +320,7 @@ const char* llama_attn_status_string(int status) {
     case LLAMA_ATTN_OK: return "ok";
     case LLAMA_ATTN_ERR_INVALID_ARG: return "invalid argument";
     case LLAMA_ATTN_ERR_UNSUPPORTED: return "unsupported shape or configuration";
-    case LLAMA_ATTN_ERR_WORKSPACE: return "decode workspace missing, misaligned or too small";
+    case LLAMA_ATTN_ERR_WORKSPACE: return "workspace or table missing, misaligned or too small";
     case LLAMA_ATTN_ERR_CUDA: return "CUDA runtime or launch failure";
     case LLAMA_ATTN_ERR_DEVICE: return "a kernel reported a device error";
     default: return "unknown status";
@@ -311,8 +340,6 @@ int llama_attn_get_device_error(cudaStream_t stream) {
 
 namespace {
 
-// bf16 prefill shared by llama_attn_prefill and llama_attn_prefill_ex: lse,
-// kcache and vcache may be null (no log-sum-exp output, no cache append).
 // Query chunks (context parallelism): q holds S rows per batch row, rows
 // [0, q_split) at global positions q_pos_a.., rows [q_split, S) at q_pos_b..;
 // k and v hold the whole sequence, Skv rows. A plain prefill is
@@ -321,58 +348,81 @@ struct QChunks {
   int Skv, q_split, q_pos_a, q_pos_b;
 };
 
-int prefill_bf16_impl(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
-                      llama_attn_bf16* out, float* lse, const int32_t* doc_offsets, int B, int S, int Hq, int Hkv,
-                      int D, float rope_theta, llama_attn_bf16* kcache, llama_attn_bf16* vcache, int Lmax,
-                      const QChunks& qc, cudaStream_t stream, bool prerotated = false) {
-  int st = check_prefill_common(q, k, v, out, B, S, Hq, Hkv, rope_theta);
-  if (st) return st;
-  const int Skv = qc.Skv;
-  if (Skv <= 0) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(B) * Skv > INT32_MAX) return LLAMA_ATTN_ERR_UNSUPPORTED;
-  if (D != 128) return LLAMA_ATTN_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if ((kcache == nullptr) != (vcache == nullptr)) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (kcache && (Lmax < S || !aligned16(kcache) || !aligned16(vcache))) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(S) * Hq * 256 >= (int64_t(1) << 40)) return LLAMA_ATTN_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(Skv) * Hkv * 256 >= (int64_t(1) << 40)) return LLAMA_ATTN_ERR_UNSUPPORTED;
-  int dev;
-  if ((st = current_device(&dev))) return st;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  DeviceCache& dc = g_cache[dev];
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-  const float2* tab = nullptr;
+// The bf16 prefill's working memory, one block: the persistent kernel's
+// work-item counter (256 B), per-token document starts (B*S int32) and the
+// rotated keys (B*Skv*Hkv*128 bf16), each part 256-byte aligned.
+struct PrefillWs {
+  size_t doc_off, krot_off, total;
+};
+PrefillWs prefill_ws_layout(int64_t B, int64_t S, int64_t Hkv) {
+  PrefillWs L;
+  L.doc_off = 256;
+  L.krot_off = L.doc_off + align256(static_cast<size_t>(B * S) * sizeof(int32_t));
+  L.total = L.krot_off + align256(static_cast<size_t>(B * S * Hkv) * 128 * 2);
+  return L;
+}
+
+// Everything the bf16 prefill launch needs besides the tensors: the RoPE
+// table (rows = positions; may be null for pre-rotated inputs without a cache
+// append) and the working memory laid out by prefill_ws_layout(B, max(S, Skv), Hkv).
+struct PrefillRes {
+  const float2* tab;
+  int tab_rows;
+  uint8_t* ws;
+};
+
+// The bf16 prefill: argument checks, then only kernel launches and a 4-byte
+// memset on `stream` (no allocation, no synchronisation). lse, kcache and
+// vcache may be null.
+int prefill_bf16_launch(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
+                        llama_attn_bf16* out, float* lse, const int32_t* doc_offsets, int B, int S, int Hq, int Hkv,
+                        llama_attn_bf16* kcache, llama_attn_bf16* vcache, int Lmax, const QChunks& qc,
+                        bool prerotated, const PrefillRes& res, int dev, cudaStream_t stream) {
+  const int Skv = qc.Skv;
   const int n_pos = S > Skv ? S : Skv;
-  if (!prerotated && (st = rope_table(dc, static_cast<double>(rope_theta), D, n_pos, stream, &tab))) return st;
+  if (!prerotated || kcache) {
+    if (res.tab == nullptr || res.tab_rows < n_pos) return LLAMA_ATTN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(res.tab) & 15u) return LLAMA_ATTN_ERR_INVALID_ARG;
+  }
+  int n_sm = 148, st;
+  if ((st = device_setup(dev, &n_sm))) return st;
+  const PrefillWs L = prefill_ws_layout(B, n_pos, Hkv);
+  int* sched = reinterpret_cast<int*>(res.ws);
+  int32_t* doc_start = doc_offsets ? reinterpret_cast<int32_t*>(res.ws + L.doc_off) : nullptr;
+  void* krot = res.ws + L.krot_off;
   const int64_t ntok = static_cast<int64_t>(B) * S;
   const int64_t nkv_tok = static_cast<int64_t>(B) * Skv;
-  const int32_t* doc_start = nullptr;
-  if (doc_offsets) {
-    if ((st = grow(reinterpret_cast<void**>(&dc.doc_start), &dc.doc_bytes, sizeof(int32_t) * ntok))) return st;
-    prof_count(1);
-    la::doc_prep_kernel<<<1, 1024, 0, stream>>>(doc_offsets, B, S, dc.doc_start);
-    LA_CUDA(cudaGetLastError());
-    doc_start = dc.doc_start;
-  }
-  const size_t kbytes = static_cast<size_t>(nkv_tok) * Hkv * 128 * 2;
-  if (!prerotated && (st = grow(&dc.krot, &dc.krot_bytes, kbytes))) return st;
-  const int64_t nvec = ntok * Hkv * 16;
-  const int64_t nvec_kv = nkv_tok * Hkv * 16;
+  const float4* tab4 = reinterpret_cast<const float4*>(res.tab);
+  // The layout passes read the offsets once per block: one wave of blocks.
+  auto stream_grid = [&](int64_t work) {
+    const int g = grid_for(work, 256);
+    return g < 8 * n_sm ? g : 8 * n_sm;
+  };
+
+  LA_CUDA(cudaMemsetAsync(sched, 0, sizeof(int), stream));
   const void* k_rot = k;  // pre-rotated keys are read as given
   if (!prerotated) {
+    // K rotation; with document offsets it also writes the per-token starts
+    const int64_t nvec_kv = nkv_tok * Hkv * 16;
     prof_count(1);
-    la::rope_rotate_rows_bf16_kernel<<<grid_for(nvec_kv, 256), 256, 0, stream>>>(
-        reinterpret_cast<const uint4*>(k), reinterpret_cast<uint4*>(dc.krot), reinterpret_cast<const float4*>(tab),
-        doc_start, Skv, Hkv, nvec_kv);
+    la::rope_rotate_rows_bf16_kernel<<<stream_grid(nvec_kv), 256, 0, stream>>>(
+        reinterpret_cast<const uint4*>(k), reinterpret_cast<uint4*>(krot), tab4, nullptr, doc_offsets, doc_start, B,
+        Skv, Hkv, nvec_kv);
     LA_CUDA(cudaGetLastError());
-    k_rot = dc.krot;
+    k_rot = krot;
+  } else if (doc_offsets) {
+    prof_count(1);
+    la::doc_prep_kernel<<<stream_grid(ntok), 256, 0, stream>>>(doc_offsets, B, S, doc_start);
+    LA_CUDA(cudaGetLastError());
   }
   if (kcache) {
+    const int64_t nvec = ntok * Hkv * 16;
     prof_count(1);
     la::kv_cache_append_kernel<<<grid_for(nvec, 256), 256, 0, stream>>>(
-        reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), reinterpret_cast<const float4*>(tab),
-        doc_start, reinterpret_cast<uint4*>(kcache), reinterpret_cast<uint4*>(vcache), S, Hkv, Lmax, nvec);
+        reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), tab4, doc_start,
+        reinterpret_cast<uint4*>(kcache), reinterpret_cast<uint4*>(vcache), S, Hkv, Lmax, nvec);
     LA_CUDA(cudaGetLastError());
   }
 
@@ -398,29 +448,97 @@ int prefill_bf16_impl(const llama_attn_bf16* q, const llama_attn_bf16* k, const 
   p.q_pos_b = qc.q_pos_b;
   p.q_rotated = prerotated ? 1 : 0;
   p.doc_start = doc_start;
-  p.rope_tab = reinterpret_cast<const float4*>(tab);
-  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  p.rope_tab = tab4;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
   p.epoch = next_epoch();
-  if (dc.sched == nullptr) LA_CUDA(cudaMalloc(&dc.sched, 256));
-  LA_CUDA(cudaMemsetAsync(dc.sched, 0, sizeof(int), stream));
-  p.sched = dc.sched;
+  p.sched = sched;
   p.lse = lse;
   const int64_t items = static_cast<int64_t>(B) * p.n_qt * p.n_hp;
   if (items > INT32_MAX) return LLAMA_ATTN_ERR_UNSUPPORTED;
-  if (!dc.prefill_attr_set) {
-    LA_CUDA(cudaFuncSetAttribute(la::pfx::prefill_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 la::pfx::SMEM_ALLOC));
-    dc.prefill_attr_set = true;
-  }
+  const int grid = static_cast<int>(items < n_sm ? items : n_sm);
   prof_count(1);
   const int pair = prof_before(stream);
-  int n_sm = 148;
-  if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
-  const int grid = static_cast<int>(items < n_sm ? items : n_sm);
   la::pfx::prefill_bf16_kernel<<<grid, la::pfx::NTHREADS, la::pfx::SMEM_ALLOC, stream>>>(tq, tk, tv, to, p);
   const cudaError_t e = cudaGetLastError();
   prof_after(pair, stream);
   return cuda_status(e);
+}
+
+// Checks shared by every bf16 prefill entry point; done before any launch.
+int check_prefill_bf16(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
+                       const llama_attn_bf16* out, const float* lse, int B, int S, int Hq, int Hkv, int D,
+                       float rope_theta, const llama_attn_bf16* kcache, const llama_attn_bf16* vcache, int Lmax,
+                       int Skv) {
+  int st = check_prefill_common(q, k, v, out, B, S, Hq, Hkv, rope_theta);
+  if (st) return st;
+  if (Skv <= 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * Skv > INT32_MAX - 1) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  if (D != 128) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if ((kcache == nullptr) != (vcache == nullptr)) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (kcache && (Lmax < S || !aligned16(kcache) || !aligned16(vcache))) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(S) * Hq * 256 >= (int64_t(1) << 40)) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(Skv) * Hkv * 256 >= (int64_t(1) << 40)) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  return LLAMA_ATTN_OK;
+}
+
+// Convenience form: the RoPE table and the working memory come from the
+// library's per-device cache (allocated, or grown, on demand: that first use
+// synchronises the device).
+int prefill_bf16_cached(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
+                        llama_attn_bf16* out, float* lse, const int32_t* doc_offsets, int B, int S, int Hq, int Hkv,
+                        int D, float rope_theta, llama_attn_bf16* kcache, llama_attn_bf16* vcache, int Lmax,
+                        const QChunks& qc, cudaStream_t stream, bool prerotated = false) {
+  int st = check_prefill_bf16(q, k, v, out, lse, B, S, Hq, Hkv, D, rope_theta, kcache, vcache, Lmax, qc.Skv);
+  if (st) return st;
+  int dev;
+  if ((st = current_device(&dev))) return st;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceCache& dc = g_cache[dev];
+  const int n_pos = S > qc.Skv ? S : qc.Skv;
+  PrefillRes res{nullptr, 0, nullptr};
+  if (!prerotated || kcache) {
+    if ((st = rope_table(dc, static_cast<double>(rope_theta), D, n_pos, stream, &res.tab))) return st;
+    res.tab_rows = n_pos;
+  }
+  const size_t need = prefill_ws_layout(B, n_pos, Hkv).total;
+  if ((st = grow(&dc.prefill_ws, &dc.prefill_ws_bytes, need))) return st;
+  res.ws = static_cast<uint8_t*>(dc.prefill_ws);
+  return prefill_bf16_launch(q, k, v, out, lse, doc_offsets, B, S, Hq, Hkv, kcache, vcache, Lmax, qc, prerotated,
+                             res, dev, stream);
+}
+
+// Caller-memory form: nothing allocated, nothing synchronised.
+int prefill_bf16_caller(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
+                        llama_attn_bf16* out, float* lse, const int32_t* doc_offsets, int B, int S, int Hq, int Hkv,
+                        int D, const void* rope_table, int rope_rows, llama_attn_bf16* kcache,
+                        llama_attn_bf16* vcache, int Lmax, const QChunks& qc, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream) {
+  int st = check_prefill_bf16(q, k, v, out, lse, B, S, Hq, Hkv, D, 500000.f, kcache, vcache, Lmax, qc.Skv);
+  if (st) return st;
+  const int n_pos = S > qc.Skv ? S : qc.Skv;
+  if (!rope_table || rope_rows < n_pos || (reinterpret_cast<uintptr_t>(rope_table) & 15u))
+    return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < prefill_ws_layout(B, n_pos, Hkv).total)
+    return LLAMA_ATTN_ERR_WORKSPACE;
+  int dev;
+  if ((st = current_device(&dev))) return st;
+  PrefillRes res{static_cast<const float2*>(rope_table), rope_rows, static_cast<uint8_t*>(workspace)};
+  std::lock_guard<std::mutex> lock(g_mutex);  // only the benchmark instrumentation is shared
+  return prefill_bf16_launch(q, k, v, out, lse, doc_offsets, B, S, Hq, Hkv, kcache, vcache, Lmax, qc, false, res,
+                             dev, stream);
+}
+
+int check_cp(int B, int Sq, int Skv, int q_pos_a, int q_split, int q_pos_b) {
+  if (B <= 0 || Sq <= 0 || Skv <= 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  constexpr int kT = la::pfx::BM;
+  if (q_split < 0 || q_split > Sq || q_pos_a < 0 || q_pos_b < 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (q_split % kT != 0 || q_pos_a % kT != 0 || q_pos_b % kT != 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(q_pos_a) + q_split > Skv) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(q_pos_b) + (Sq - q_split) > Skv) return LLAMA_ATTN_ERR_INVALID_ARG;
+  return LLAMA_ATTN_OK;
 }
 
 }  // namespace
@@ -430,36 +548,72 @@ extern "C" {
 int llama_attn_prefill(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
                        llama_attn_bf16* out, const int32_t* doc_offsets, int B, int S, int Hq, int Hkv, int D,
                        float rope_theta, cudaStream_t stream) {
-  return prefill_bf16_impl(q, k, v, out, nullptr, doc_offsets, B, S, Hq, Hkv, D, rope_theta, nullptr, nullptr, 0,
-                           QChunks{S, S, 0, 0}, stream);
+  return prefill_bf16_cached(q, k, v, out, nullptr, doc_offsets, B, S, Hq, Hkv, D, rope_theta, nullptr, nullptr, 0,
+                             QChunks{S, S, 0, 0}, stream);
 }
 
 int llama_attn_prefill_ex(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
                           llama_attn_bf16* out, float* lse, const int32_t* doc_offsets, int B, int S, int Hq,
                           int Hkv, int D, float rope_theta, llama_attn_bf16* kcache, llama_attn_bf16* vcache,
                           int Lmax, cudaStream_t stream) {
-  return prefill_bf16_impl(q, k, v, out, lse, doc_offsets, B, S, Hq, Hkv, D, rope_theta, kcache, vcache, Lmax,
-                           QChunks{S, S, 0, 0}, stream);
+  return prefill_bf16_cached(q, k, v, out, lse, doc_offsets, B, S, Hq, Hkv, D, rope_theta, kcache, vcache, Lmax,
+                             QChunks{S, S, 0, 0}, stream);
 }
 
 int llama_attn_prefill_cp(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
                           llama_attn_bf16* out, float* lse, int B, int Sq, int Skv, int Hq, int Hkv, int D,
                           int q_pos_a, int q_split, int q_pos_b, float rope_theta, cudaStream_t stream) {
-  if (B <= 0 || Sq <= 0 || Skv <= 0) return LLAMA_ATTN_ERR_INVALID_ARG;
-  constexpr int kT = la::pfx::BM;
-  if (q_split < 0 || q_split > Sq || q_pos_a < 0 || q_pos_b < 0) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (q_split % kT != 0 || q_pos_a % kT != 0 || q_pos_b % kT != 0) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(q_pos_a) + q_split > Skv) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(q_pos_b) + (Sq - q_split) > Skv) return LLAMA_ATTN_ERR_INVALID_ARG;
-  return prefill_bf16_impl(q, k, v, out, lse, nullptr, B, Sq, Hq, Hkv, D, rope_theta, nullptr, nullptr, 0,
-                           QChunks{Skv, q_split, q_pos_a, q_pos_b}, stream);
+  const int st = check_cp(B, Sq, Skv, q_pos_a, q_split, q_pos_b);
+  if (st) return st;
+  return prefill_bf16_cached(q, k, v, out, lse, nullptr, B, Sq, Hq, Hkv, D, rope_theta, nullptr, nullptr, 0,
+                             QChunks{Skv, q_split, q_pos_a, q_pos_b}, stream);
 }
 
 int llama_attn_prefill_rotated(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
                                llama_attn_bf16* out, float* lse, const int32_t* doc_offsets, int B, int S, int Hq,
                                int Hkv, int D, cudaStream_t stream) {
-  return prefill_bf16_impl(q, k, v, out, lse, doc_offsets, B, S, Hq, Hkv, D, 500000.f, nullptr, nullptr, 0,
-                           QChunks{S, S, 0, 0}, stream, true);
+  return prefill_bf16_cached(q, k, v, out, lse, doc_offsets, B, S, Hq, Hkv, D, 500000.f, nullptr, nullptr, 0,
+                             QChunks{S, S, 0, 0}, stream, true);
+}
+
+size_t llama_attn_rope_table_size(int maxpos, int D) {
+  if (maxpos <= 0 || D < 2 || D > 128 || (D % 2) != 0) return 0;
+  return static_cast<size_t>(maxpos) * (D / 2) * sizeof(float2);
+}
+
+int llama_attn_rope_table_build(void* table, size_t table_bytes, int maxpos, int D, float rope_theta,
+                                cudaStream_t stream) {
+  const size_t need = llama_attn_rope_table_size(maxpos, D);
+  if (!table || need == 0 || (reinterpret_cast<uintptr_t>(table) & 15u)) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (!(rope_theta > 0.f) || !std::isfinite(rope_theta)) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (table_bytes < need) return LLAMA_ATTN_ERR_WORKSPACE;
+  la::rope_table_kernel<<<grid_for(static_cast<int64_t>(maxpos) * (D / 2), 256), 256, 0, stream>>>(
+      static_cast<float2*>(table), maxpos, D, static_cast<double>(rope_theta));
+  return cuda_status(cudaGetLastError());
+}
+
+size_t llama_attn_prefill_workspace_size(int B, int S, int Hkv, int D) {
+  if (B <= 0 || S <= 0 || Hkv <= 0 || D != 128) return 0;
+  return prefill_ws_layout(B, S, Hkv).total;
+}
+
+int llama_attn_prefill_ws(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
+                          llama_attn_bf16* out, float* lse, const int32_t* doc_offsets, int B, int S, int Hq,
+                          int Hkv, int D, const void* rope_table, int rope_rows, llama_attn_bf16* kcache,
+                          llama_attn_bf16* vcache, int Lmax, void* workspace, size_t workspace_bytes,
+                          cudaStream_t stream) {
+  return prefill_bf16_caller(q, k, v, out, lse, doc_offsets, B, S, Hq, Hkv, D, rope_table, rope_rows, kcache, vcache,
+                             Lmax, QChunks{S, S, 0, 0}, workspace, workspace_bytes, stream);
+}
+
+int llama_attn_prefill_cp_ws(const llama_attn_bf16* q, const llama_attn_bf16* k, const llama_attn_bf16* v,
+                             llama_attn_bf16* out, float* lse, int B, int Sq, int Skv, int Hq, int Hkv, int D,
+                             int q_pos_a, int q_split, int q_pos_b, const void* rope_table, int rope_rows,
+                             void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const int st = check_cp(B, Sq, Skv, q_pos_a, q_split, q_pos_b);
+  if (st) return st;
+  return prefill_bf16_caller(q, k, v, out, lse, nullptr, B, Sq, Hq, Hkv, D, rope_table, rope_rows, nullptr, nullptr,
+                             0, QChunks{Skv, q_split, q_pos_a, q_pos_b}, workspace, workspace_bytes, stream);
 }
 
 int llama_attn_quantize_e4m3(const llama_attn_bf16* x, int64_t n, uint8_t* y, float* scale, cudaStream_t stream) {
@@ -504,11 +658,14 @@ int llama_attn_qkv_fp8_rope(const uint8_t* x, const float* s_x, const uint8_t* w
   DeviceCache& dc = g_cache[dev];
   const float2* tab = nullptr;
   if ((st = rope_table(dc, static_cast<double>(rope_theta), D, S, stream, &tab))) return st;
+  int n_sm = 148;
+  if ((st = device_setup(dev, &n_sm))) return st;
   const int32_t* doc_start = nullptr;
   if (doc_offsets) {
     if ((st = grow(reinterpret_cast<void**>(&dc.doc_start), &dc.doc_bytes, sizeof(int32_t) * M))) return st;
     prof_count(1);
-    la::doc_prep_kernel<<<1, 1024, 0, stream>>>(doc_offsets, B, S, dc.doc_start);
+    const int g = grid_for(M, 256);
+    la::doc_prep_kernel<<<g < 8 * n_sm ? g : 8 * n_sm, 256, 0, stream>>>(doc_offsets, B, S, dc.doc_start);
     LA_CUDA(cudaGetLastError());
     doc_start = dc.doc_start;
   }
@@ -539,13 +696,6 @@ int llama_attn_qkv_fp8_rope(const uint8_t* x, const float* s_x, const uint8_t* w
   p.epoch = next_epoch();
   const int64_t tiles = static_cast<int64_t>(p.n_mt) * p.n_nt;
   if (tiles > INT32_MAX) return LLAMA_ATTN_ERR_UNSUPPORTED;
-  if (!dc.qkv_attr_set) {
-    LA_CUDA(cudaFuncSetAttribute(la::q8::qkv_fp8_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 la::q8::SMEM_ALLOC));
-    dc.qkv_attr_set = true;
-  }
-  int n_sm = 148;
-  if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0) n_sm = 148;
   const int grid = static_cast<int>(tiles < n_sm ? tiles : n_sm);
   prof_count(1);
   const int pair = prof_before(stream);
@@ -568,11 +718,14 @@ int llama_attn_prefill_f32(const float* q, const float* k, const float* v, float
   const float2* tab = nullptr;
   if ((st = rope_table(dc, static_cast<double>(rope_theta), D, S, stream, &tab))) return st;
   const int64_t ntok = static_cast<int64_t>(B) * S;
+  int n_sm = 148;
+  if ((st = device_setup(dev, &n_sm))) return st;
   const int32_t* doc_start = nullptr;
   if (doc_offsets) {
     if ((st = grow(reinterpret_cast<void**>(&dc.doc_start), &dc.doc_bytes, sizeof(int32_t) * ntok))) return st;
     prof_count(1);
-    la::doc_prep_kernel<<<1, 1024, 0, stream>>>(doc_offsets, B, S, dc.doc_start);
+    const int g = grid_for(ntok, 256);
+    la::doc_prep_kernel<<<g < 8 * n_sm ? g : 8 * n_sm, 256, 0, stream>>>(doc_offsets, B, S, dc.doc_start);
     LA_CUDA(cudaGetLastError());
     doc_start = dc.doc_start;
   }
@@ -602,145 +755,30 @@ size_t llama_attn_decode_workspace_size(int B, int Hq, int Lmax, int D) {
   return ((o_bytes + lse_bytes + 255) / 256) * 256;
 }
 
-int llama_attn_decode(const llama_attn_bf16* q, const llama_attn_bf16* kcache, const llama_attn_bf16* vcache,
-                      const int32_t* cache_lens, llama_attn_bf16* out, int B, int Hq, int Hkv, int D, int Lmax,
-                      float rope_theta, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  if (!q || !kcache || !vcache || !cache_lens || !out) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lmax <= 0 || Hq % Hkv != 0) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (!(rope_theta > 0.f) || !std::isfinite(rope_theta)) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (D != 128 || Hq / Hkv > 16) return LLAMA_ATTN_ERR_UNSUPPORTED;
-  if (B > 65535 || Hkv > 65535 || B * Hq > INT32_MAX / 2) return LLAMA_ATTN_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(B) * Hkv * Lmax >= INT32_MAX) return LLAMA_ATTN_ERR_UNSUPPORTED;
-  if (!aligned16(kcache) || !aligned16(vcache) || !aligned16(q) || !aligned16(out)) return LLAMA_ATTN_ERR_INVALID_ARG;
-  const size_t need = llama_attn_decode_workspace_size(B, Hq, Lmax, D);
-  if (!workspace || !aligned16(workspace) || workspace_bytes < need) return LLAMA_ATTN_ERR_WORKSPACE;
-  int dev, st;
-  if ((st = current_device(&dev))) return st;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  DeviceCache& dc = g_cache[dev];
-  const float2* tab = nullptr;
-  if ((st = rope_table(dc, static_cast<double>(rope_theta), D, Lmax + 1, stream, &tab))) return st;
+}  // extern "C"
 
-  CUtensorMap tk, tv;
-  const int64_t rows = static_cast<int64_t>(B) * Hkv * Lmax;
-  if ((st = tmap_rows(&tk, kcache, rows))) return st;
-  if ((st = tmap_rows(&tv, vcache, rows))) return st;
+namespace {
 
-  la::dec::Params p;
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.G = Hq / Hkv;
-  p.Lmax = Lmax;
-  p.nchunk = (Lmax + la::dec::CHUNK - 1) / la::dec::CHUNK;
-  p.lens = cache_lens;
-  p.q = q;
-  p.rope_tab = reinterpret_cast<const float4*>(tab);
-  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-  p.epoch = next_epoch();
-  p.rope_theta = static_cast<double>(rope_theta);
-  const size_t slots = static_cast<size_t>(B) * Hq * p.nchunk;
-  p.part_o = static_cast<float*>(workspace);
-  p.part_lse = p.part_o + slots * 128;
-  if (!dc.decode_attr_set) {
-    LA_CUDA(cudaFuncSetAttribute(la::dec::decode_split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 la::dec::SMEM_ALLOC));
-    dc.decode_attr_set = true;
-  }
-  const dim3 grid(p.nchunk, Hkv, B);
-  prof_count(2);
-  const int pair = prof_before(stream);
-  la::dec::decode_split_kernel<false><<<grid, la::dec::NTHREADS, la::dec::SMEM_ALLOC, stream>>>(tk, tv, p);
-  const cudaError_t e = cudaGetLastError();
-  prof_after(pair, stream);
-  if (e != cudaSuccess) return LLAMA_ATTN_ERR_CUDA;
-  la::dec::decode_combine_kernel<<<B * Hq, 128, 0, stream>>>(p.part_o, p.part_lse, cache_lens, out, Hq, Lmax,
-                                                            p.nchunk);
-  return cuda_status(cudaGetLastError());
-}
-
-int llama_attn_decode_noalloc(const llama_attn_bf16* q, const llama_attn_bf16* kcache,
-                              const llama_attn_bf16* vcache, const int32_t* cache_lens, llama_attn_bf16* out, int B,
-                              int Hq, int Hkv, int D, int Lmax, float rope_theta, cudaStream_t stream) {
-  if (!q || !kcache || !vcache || !cache_lens || !out) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lmax <= 0 || Hq % Hkv != 0) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (!(rope_theta > 0.f) || !std::isfinite(rope_theta)) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (D != 128 || Hq / Hkv > 16) return LLAMA_ATTN_ERR_UNSUPPORTED;
-  if (B > 65535 || Hkv > 65535 || B * Hq > INT32_MAX / 2) return LLAMA_ATTN_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(B) * Hkv * Lmax >= INT32_MAX) return LLAMA_ATTN_ERR_UNSUPPORTED;
-  if (!aligned16(kcache) || !aligned16(vcache) || !aligned16(q) || !aligned16(out)) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (llama_attn_decode_workspace_size(B, Hq, Lmax, D) > kNoAllocScratchBytes) return LLAMA_ATTN_ERR_WORKSPACE;
-  int dev, st;
-  if ((st = current_device(&dev))) return st;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_noalloc_scratch_addr[dev] == nullptr) {
-    void* addr = nullptr;
-    if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || addr == nullptr) return LLAMA_ATTN_ERR_CUDA;
-    g_noalloc_scratch_addr[dev] = addr;
-  }
-  if (!g_noalloc_attr_set[dev]) {
-    LA_CUDA(cudaFuncSetAttribute(la::dec::decode_split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 la::dec::SMEM_ALLOC_SELF_TABLE));
-    g_noalloc_attr_set[dev] = true;
-  }
-  CUtensorMap tk, tv;
-  const int64_t rows = static_cast<int64_t>(B) * Hkv * Lmax;
-  if ((st = tmap_rows(&tk, kcache, rows))) return st;
-  if ((st = tmap_rows(&tv, vcache, rows))) return st;
-
-  la::dec::Params p;
-  p.B = B;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.G = Hq / Hkv;
-  p.Lmax = Lmax;
-  p.nchunk = (Lmax + la::dec::CHUNK - 1) / la::dec::CHUNK;
-  p.lens = cache_lens;
-  p.q = q;
-  p.rope_tab = nullptr;
-  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
-  p.epoch = next_epoch();
-  p.rope_theta = static_cast<double>(rope_theta);
-  const size_t slots = static_cast<size_t>(B) * Hq * p.nchunk;
-  p.part_o = static_cast<float*>(g_noalloc_scratch_addr[dev]);
-  p.part_lse = p.part_o + slots * 128;
-  const dim3 grid(p.nchunk, Hkv, B);
-  la::dec::decode_split_kernel<true><<<grid, la::dec::NTHREADS, la::dec::SMEM_ALLOC_SELF_TABLE, stream>>>(tk, tv, p);
-  LA_CUDA(cudaGetLastError());
-  la::dec::decode_combine_kernel<<<B * Hq, 128, 0, stream>>>(p.part_o, p.part_lse, cache_lens, out, Hq, Lmax,
-                                                            p.nchunk);
-  return cuda_status(cudaGetLastError());
-}
-
-int llama_attn_decode_paged(const llama_attn_bf16* q, const llama_attn_bf16* kpages, const llama_attn_bf16* vpages,
-                            const int32_t* block_table, const int32_t* cache_lens, llama_attn_bf16* out, int B,
-                            int Hq, int Hkv, int D, int page_size, int max_blocks, int n_pages, float rope_theta,
-                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  if (!q || !kpages || !vpages || !block_table || !cache_lens || !out) return LLAMA_ATTN_ERR_INVALID_ARG;
+// Argument checks shared by the decode entry points (before any launch).
+int check_decode(const void* q, const void* kc, const void* vc, const int32_t* lens, const void* out, int B, int Hq,
+                 int Hkv, int D, float rope_theta) {
+  if (!q || !kc || !vc || !lens || !out) return LLAMA_ATTN_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (page_size <= 0 || max_blocks <= 0 || n_pages <= 0) return LLAMA_ATTN_ERR_INVALID_ARG;
   if (!(rope_theta > 0.f) || !std::isfinite(rope_theta)) return LLAMA_ATTN_ERR_INVALID_ARG;
-  if (D != 128 || Hq / Hkv > 16 || page_size % la::dec::ROWS != 0) return LLAMA_ATTN_ERR_UNSUPPORTED;
-  if (B > 65535 || Hkv > 65535 || B * Hq > INT32_MAX / 2) return LLAMA_ATTN_ERR_UNSUPPORTED;
-  const int64_t Lmax64 = static_cast<int64_t>(max_blocks) * page_size;
-  if (Lmax64 >= INT32_MAX || static_cast<int64_t>(n_pages) * Hkv * page_size >= INT32_MAX - page_size)
+  if (D != 128 || Hq / Hkv > 16) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  // grid (chunks, Hkv, B) and the combine's B * Hq blocks
+  if (B > 65535 || Hkv > 65535 || Hq > 65535 || static_cast<int64_t>(B) * Hq > INT32_MAX / 2)
     return LLAMA_ATTN_ERR_UNSUPPORTED;
-  const int Lmax = static_cast<int>(Lmax64);
-  if (!aligned16(kpages) || !aligned16(vpages) || !aligned16(q) || !aligned16(out)) return LLAMA_ATTN_ERR_INVALID_ARG;
-  const size_t need = llama_attn_decode_workspace_size(B, Hq, Lmax, D);
-  if (!workspace || !aligned16(workspace) || workspace_bytes < need) return LLAMA_ATTN_ERR_WORKSPACE;
-  int dev, st;
-  if ((st = current_device(&dev))) return st;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  DeviceCache& dc = g_cache[dev];
-  const float2* tab = nullptr;
-  if ((st = rope_table(dc, static_cast<double>(rope_theta), D, Lmax + 1, stream, &tab))) return st;
+  if (!aligned16(kc) || !aligned16(vc) || !aligned16(q) || !aligned16(out)) return LLAMA_ATTN_ERR_INVALID_ARG;
+  return LLAMA_ATTN_OK;
+}
 
-  CUtensorMap tk, tv;
-  const int64_t rows = static_cast<int64_t>(n_pages) * Hkv * page_size;
-  if ((st = tmap_rows(&tk, kpages, rows))) return st;
-  if ((st = tmap_rows(&tv, vpages, rows))) return st;
-
+// Split-KV partial attention and the log-sum-exp combine, on `stream`, with
+// the partials in `part` (llama_attn_decode_workspace_size bytes). Paged when
+// block_table is not null. Launches only: no allocation, no synchronisation.
+int decode_launch(const llama_attn_bf16* q, const CUtensorMap& tk, const CUtensorMap& tv, const int32_t* lens,
+                  llama_attn_bf16* out, int B, int Hq, int Hkv, int Lmax, float rope_theta, const int32_t* block_table,
+                  int page_size, int max_blocks, int n_pages, void* part, cudaStream_t stream) {
   la::dec::Params p;
   p.B = B;
   p.Hq = Hq;
@@ -748,10 +786,9 @@ int llama_attn_decode_paged(const llama_attn_bf16* q, const llama_attn_bf16* kpa
   p.G = Hq / Hkv;
   p.Lmax = Lmax;
   p.nchunk = (Lmax + la::dec::CHUNK - 1) / la::dec::CHUNK;
-  p.lens = cache_lens;
+  p.lens = lens;
   p.q = q;
-  p.rope_tab = reinterpret_cast<const float4*>(tab);
-  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
   p.epoch = next_epoch();
   p.rope_theta = static_cast<double>(rope_theta);
   p.block_table = block_table;
@@ -759,23 +796,95 @@ int llama_attn_decode_paged(const llama_attn_bf16* q, const llama_attn_bf16* kpa
   p.max_blocks = max_blocks;
   p.n_pages = n_pages;
   const size_t slots = static_cast<size_t>(B) * Hq * p.nchunk;
-  p.part_o = static_cast<float*>(workspace);
+  p.part_o = static_cast<float*>(part);
   p.part_lse = p.part_o + slots * 128;
-  if (!dc.decode_paged_attr_set) {
-    LA_CUDA(cudaFuncSetAttribute(la::dec::decode_split_kernel<false, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, la::dec::SMEM_ALLOC));
-    dc.decode_paged_attr_set = true;
-  }
   const dim3 grid(p.nchunk, Hkv, B);
   prof_count(2);
   const int pair = prof_before(stream);
-  la::dec::decode_split_kernel<false, true><<<grid, la::dec::NTHREADS, la::dec::SMEM_ALLOC, stream>>>(tk, tv, p);
+  if (block_table)
+    la::dec::decode_split_kernel<true><<<grid, la::dec::NTHREADS, la::dec::SMEM_ALLOC, stream>>>(tk, tv, p);
+  else
+    la::dec::decode_split_kernel<false><<<grid, la::dec::NTHREADS, la::dec::SMEM_ALLOC, stream>>>(tk, tv, p);
   const cudaError_t e = cudaGetLastError();
   prof_after(pair, stream);
   if (e != cudaSuccess) return LLAMA_ATTN_ERR_CUDA;
-  la::dec::decode_combine_kernel<<<B * Hq, 128, 0, stream>>>(p.part_o, p.part_lse, cache_lens, out, Hq, Lmax,
-                                                            p.nchunk);
+  la::dec::decode_combine_kernel<<<B * Hq, 128, 0, stream>>>(p.part_o, p.part_lse, lens, out, Hq, Lmax, p.nchunk);
   return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+extern "C" {
+
+int llama_attn_decode(const llama_attn_bf16* q, const llama_attn_bf16* kcache, const llama_attn_bf16* vcache,
+                      const int32_t* cache_lens, llama_attn_bf16* out, int B, int Hq, int Hkv, int D, int Lmax,
+                      float rope_theta, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  int st = check_decode(q, kcache, vcache, cache_lens, out, B, Hq, Hkv, D, rope_theta);
+  if (st) return st;
+  if (Lmax <= 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * Hkv * Lmax >= INT32_MAX) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  const size_t need = llama_attn_decode_workspace_size(B, Hq, Lmax, D);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < need) return LLAMA_ATTN_ERR_WORKSPACE;
+  int dev;
+  if ((st = current_device(&dev))) return st;
+  if ((st = device_setup(dev, nullptr))) return st;
+  CUtensorMap tk, tv;
+  const int64_t rows = static_cast<int64_t>(B) * Hkv * Lmax;
+  if ((st = tmap_rows(&tk, kcache, rows))) return st;
+  if ((st = tmap_rows(&tv, vcache, rows))) return st;
+  std::lock_guard<std::mutex> lock(g_mutex);  // only the benchmark instrumentation is shared
+  return decode_launch(q, tk, tv, cache_lens, out, B, Hq, Hkv, Lmax, rope_theta, nullptr, 0, 0, 0, workspace, stream);
+}
+
+int llama_attn_decode_noalloc(const llama_attn_bf16* q, const llama_attn_bf16* kcache,
+                              const llama_attn_bf16* vcache, const int32_t* cache_lens, llama_attn_bf16* out, int B,
+                              int Hq, int Hkv, int D, int Lmax, float rope_theta, cudaStream_t stream) {
+  int st = check_decode(q, kcache, vcache, cache_lens, out, B, Hq, Hkv, D, rope_theta);
+  if (st) return st;
+  if (Lmax <= 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * Hkv * Lmax >= INT32_MAX) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  if (llama_attn_decode_workspace_size(B, Hq, Lmax, D) > kNoAllocScratchBytes) return LLAMA_ATTN_ERR_WORKSPACE;
+  int dev;
+  if ((st = current_device(&dev))) return st;
+  if ((st = device_setup(dev, nullptr))) return st;
+  CUtensorMap tk, tv;
+  const int64_t rows = static_cast<int64_t>(B) * Hkv * Lmax;
+  if ((st = tmap_rows(&tk, kcache, rows))) return st;
+  if ((st = tmap_rows(&tv, vcache, rows))) return st;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_noalloc_scratch_addr[dev] == nullptr) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || addr == nullptr) return LLAMA_ATTN_ERR_CUDA;
+    g_noalloc_scratch_addr[dev] = addr;
+  }
+  return decode_launch(q, tk, tv, cache_lens, out, B, Hq, Hkv, Lmax, rope_theta, nullptr, 0, 0, 0,
+                       g_noalloc_scratch_addr[dev], stream);
+}
+
+int llama_attn_decode_paged(const llama_attn_bf16* q, const llama_attn_bf16* kpages, const llama_attn_bf16* vpages,
+                            const int32_t* block_table, const int32_t* cache_lens, llama_attn_bf16* out, int B,
+                            int Hq, int Hkv, int D, int page_size, int max_blocks, int n_pages, float rope_theta,
+                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  int st = check_decode(q, kpages, vpages, cache_lens, out, B, Hq, Hkv, D, rope_theta);
+  if (st) return st;
+  if (!block_table || page_size <= 0 || max_blocks <= 0 || n_pages <= 0) return LLAMA_ATTN_ERR_INVALID_ARG;
+  if (page_size % la::dec::ROWS != 0) return LLAMA_ATTN_ERR_UNSUPPORTED;
+  const int64_t Lmax64 = static_cast<int64_t>(max_blocks) * page_size;
+  if (Lmax64 >= INT32_MAX || static_cast<int64_t>(n_pages) * Hkv * page_size >= INT32_MAX - page_size)
+    return LLAMA_ATTN_ERR_UNSUPPORTED;
+  const int Lmax = static_cast<int>(Lmax64);
+  const size_t need = llama_attn_decode_workspace_size(B, Hq, Lmax, D);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < need) return LLAMA_ATTN_ERR_WORKSPACE;
+  int dev;
+  if ((st = current_device(&dev))) return st;
+  if ((st = device_setup(dev, nullptr))) return st;
+  CUtensorMap tk, tv;
+  const int64_t rows = static_cast<int64_t>(n_pages) * Hkv * page_size;
+  if ((st = tmap_rows(&tk, kpages, rows))) return st;
+  if ((st = tmap_rows(&tv, vpages, rows))) return st;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  return decode_launch(q, tk, tv, cache_lens, out, B, Hq, Hkv, Lmax, rope_theta, block_table, page_size, max_blocks,
+                       n_pages, workspace, stream);
 }
 
 }  // extern "C"

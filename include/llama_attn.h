@@ -25,14 +25,25 @@
  * Conventions for every call:
  *   - All tensor pointers are DEVICE pointers to contiguous memory, owned by
  *     the caller. bf16 tensors are passed as raw 16-bit patterns.
- *   - Calls are asynchronous on `stream` (NULL = legacy default stream) and do
- *     not synchronise the host, except that the first use of a (device, theta,
- *     D) RoPE table, or a request that outgrows a cached table or scratch
- *     buffer, allocates device memory (cudaMalloc) before enqueueing work.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream).
+ *   - Two forms of the bf16 prefill. The *_ws entry points take every buffer
+ *     from the caller (a RoPE table built once by llama_attn_rope_table_build
+ *     and a workspace of llama_attn_prefill_workspace_size bytes): they only
+ *     enqueue kernels and a 4-byte memset, never allocate and never
+ *     synchronise. The convenience entry points (llama_attn_prefill, _ex, _cp,
+ *     _rotated, and the fp32 and FP8 calls) keep the table and the workspace
+ *     in a library-owned per-device cache instead: the first use of a
+ *     (device, theta, D) table, or a request larger than the cached buffers,
+ *     allocates device memory and synchronises the device before enqueueing
+ *     work; later calls of the same or smaller sizes do neither.
+ *   - The decode calls never allocate or synchronise: the caller passes the
+ *     workspace and the query's RoPE row is formed inside the kernel.
  *   - Arguments are checked on the host before anything is launched; a
  *     failed check returns a negative status and launches nothing.
- *   - The library keeps per-device caches (RoPE tables, scratch); calls from
- *     several host threads at once are not supported.
+ *   - The convenience calls share their per-device caches: calls from several
+ *     host threads at once are serialised by a lock, and two calls whose
+ *     kernels can overlap on the GPU (different streams, no ordering) must not
+ *     both use the cache. Calls with caller-owned memory share nothing.
  *   - No C++ exception crosses this interface.
  */
 #ifndef LLAMA_ATTN_H
@@ -75,8 +86,9 @@ typedef enum {
  *     the output is then unspecified and the device error word is set to
  *     LLAMA_ATTN_DEVERR_DOC_OFFSETS.
  *   B, S >= 1; Hq, Hkv >= 1 with Hq % Hkv == 0; D == 128; rope_theta > 0.
- *   Scratch: the call keeps a library-owned rotated copy of k (B*S*Hkv*D bf16)
- *   and per-token document data, grown on demand.
+ *   Working memory (a rotated copy of k, B*S*Hkv*D bf16, and the per-token
+ *   document starts) comes from the library's per-device cache; see
+ *   llama_attn_prefill_ws for the form that takes it from the caller.
  */
 int llama_attn_prefill(const llama_attn_bf16 *q, const llama_attn_bf16 *k,
                        const llama_attn_bf16 *v, llama_attn_bf16 *out,
@@ -137,6 +149,68 @@ int llama_attn_prefill_cp(const llama_attn_bf16 *q, const llama_attn_bf16 *k,
                           const llama_attn_bf16 *v, llama_attn_bf16 *out, float *lse, int B,
                           int Sq, int Skv, int Hq, int Hkv, int D, int q_pos_a, int q_split,
                           int q_pos_b, float rope_theta, cudaStream_t stream);
+
+/*
+ * Caller-owned RoPE table for the *_ws entry points: rows 0 .. maxpos-1, row
+ * p holding (cos(p theta_k), sin(p theta_k)) as two floats for k = 0 ..
+ * D/2-1, theta_k = rope_theta^(-2k/D) (the frequencies of "Llama 3.1
+ * Architecture ...", "Context Expansion", "High Base Frequency"). The angle
+ * p theta_k is formed and reduced in float64 and only cos and sin are rounded
+ * to float32 (a float32 product is off by ~4e-3 rad at p ~ 1.3e5).
+ *
+ * llama_attn_rope_table_size returns the bytes for maxpos rows (0 for
+ * maxpos < 1 or D not even in [2, 128]). llama_attn_rope_table_build writes
+ * the table into `table` (device, 16-byte aligned, table_bytes >= that size,
+ * else LLAMA_ATTN_ERR_WORKSPACE) with one kernel on `stream`. Build it once
+ * per (theta, D) and reuse it: for 128K positions and D = 128 it is 64 MiB.
+ */
+size_t llama_attn_rope_table_size(int maxpos, int D);
+int llama_attn_rope_table_build(void *table, size_t table_bytes, int maxpos, int D,
+                                float rope_theta, cudaStream_t stream);
+
+/*
+ * Bytes of device workspace the bf16 prefill needs with caller-owned memory:
+ * a 256-byte work-item counter, the per-token document starts (B*S int32) and
+ * the rotated keys (B*S*Hkv*D bf16), each part 256-byte aligned. S is the
+ * number of key rows per batch row (Skv for llama_attn_prefill_cp_ws). Returns
+ * 0 for invalid sizes (D must be 128).
+ */
+size_t llama_attn_prefill_workspace_size(int B, int S, int Hkv, int D);
+
+/*
+ * llama_attn_prefill_ex with caller-owned memory: the same attention, LSE and
+ * optional KV-cache append, with
+ *
+ *   rope_table, rope_rows  a table from llama_attn_rope_table_build (D = 128,
+ *          the base of its build is the rope_theta of the computation), 16-byte
+ *          aligned, rope_rows >= S rows (else LLAMA_ATTN_ERR_INVALID_ARG)
+ *   workspace, workspace_bytes  device memory, 256-byte aligned, at least
+ *          llama_attn_prefill_workspace_size(B, S, Hkv, D) bytes (else
+ *          LLAMA_ATTN_ERR_WORKSPACE, before anything is launched); its contents
+ *          need no initialisation and are overwritten.
+ *
+ * The call only enqueues kernels and a 4-byte memset on `stream`: no
+ * allocation, no synchronisation. Two calls whose kernels can overlap on the
+ * GPU must not share a workspace. Other arguments and errors as for
+ * llama_attn_prefill_ex.
+ */
+int llama_attn_prefill_ws(const llama_attn_bf16 *q, const llama_attn_bf16 *k,
+                          const llama_attn_bf16 *v, llama_attn_bf16 *out, float *lse,
+                          const int32_t *doc_offsets, int B, int S, int Hq, int Hkv, int D,
+                          const void *rope_table, int rope_rows, llama_attn_bf16 *kcache,
+                          llama_attn_bf16 *vcache, int Lmax, void *workspace,
+                          size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * llama_attn_prefill_cp with caller-owned memory: rope_rows >= Skv, workspace
+ * of llama_attn_prefill_workspace_size(B, Skv, Hkv, D) bytes; otherwise as
+ * llama_attn_prefill_cp and llama_attn_prefill_ws.
+ */
+int llama_attn_prefill_cp_ws(const llama_attn_bf16 *q, const llama_attn_bf16 *k,
+                             const llama_attn_bf16 *v, llama_attn_bf16 *out, float *lse, int B,
+                             int Sq, int Skv, int Hq, int Hkv, int D, int q_pos_a, int q_split,
+                             int q_pos_b, const void *rope_table, int rope_rows, void *workspace,
+                             size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Prefill on queries and keys that are already rotated (for example by
@@ -226,6 +300,9 @@ size_t llama_attn_decode_workspace_size(int B, int Hq, int Lmax, int D);
  *   workspace: device memory of at least
  *   llama_attn_decode_workspace_size(B, Hq, Lmax, D) bytes, 16-byte aligned,
  *   owned by the caller; its contents need no initialisation.
+ *   The (cos, sin) row of position cache_lens[b] is formed in the kernel
+ *   (float64 angle), so the call reads no table, allocates nothing and does
+ *   not synchronise.
  */
 int llama_attn_decode(const llama_attn_bf16 *q, const llama_attn_bf16 *kcache,
                       const llama_attn_bf16 *vcache, const int32_t *cache_lens,
@@ -261,10 +338,10 @@ int llama_attn_decode_paged(const llama_attn_bf16 *q, const llama_attn_bf16 *kpa
 
 /*
  * llama_attn_decode without a caller-supplied workspace and without any
- * device allocation, for callers that cannot allocate device memory: code
- * that runs inside a CUDA graph capture, under an allocator that owns all of
- * device memory, or in a host without access to cudaMalloc. Nothing on the
- * pages corresponds to it; it exists only for such callers.
+ * device allocation, for callers that cannot allocate device memory: a host
+ * whose allocator owns all of device memory, or code running where
+ * cudaMalloc is not allowed. Nothing on the pages corresponds to it; it exists
+ * only for such callers.
  *
  * Same arguments, layouts, results and error codes as llama_attn_decode, minus
  * the workspace. The split-KV partials live in one fixed 72 MiB device array
@@ -281,7 +358,9 @@ int llama_attn_decode_paged(const llama_attn_bf16 *q, const llama_attn_bf16 *kpa
  * last call's contents; nothing in it needs to start at zero, because every
  * partial is written before it is read within a call. Calls whose kernels can
  * overlap on the GPU (different streams, no ordering between them) race on
- * the array: order them, e.g. on one stream.
+ * the array: order them, e.g. on one stream. If a call's kernels give up a
+ * bounded wait (LLAMA_ATTN_DEVERR_TIMEOUT in the device error word), the
+ * output of that call is undefined.
  */
 int llama_attn_decode_noalloc(const llama_attn_bf16 *q, const llama_attn_bf16 *kcache,
                               const llama_attn_bf16 *vcache, const int32_t *cache_lens,

@@ -131,6 +131,70 @@ def test_fp8_entries_reject(lib):
     assert r(FAKE, FAKE, FAKE, FAKE, None, None, 1, 128, 8, 2, 64, None) == UNSUPPORTED
 
 
+def test_prefill_workspace_and_table_sizes(lib):
+    ws = lib.llama_attn_prefill_workspace_size
+    assert ws(0, 128, 8, 128) == 0 and ws(1, 128, 8, 64) == 0 and ws(1, 0, 8, 128) == 0
+    B, S, Hkv = 4, 8192, 8
+    n = ws(B, S, Hkv, 128)
+    # counter (256 B) + document starts (B*S int32) + rotated keys (B*S*Hkv*128 bf16), each 256-aligned
+    assert n == 256 + B * S * 4 + B * S * Hkv * 256
+    assert ws(1, 1, 1, 128) == 256 + 256 + 256
+    ts = lib.llama_attn_rope_table_size
+    assert ts(131072, 128) == 131072 * 64 * 8
+    assert ts(0, 128) == 0 and ts(16, 7) == 0 and ts(16, 130) == 0
+
+
+T16 = ctypes.c_void_p(4096 * 16)  # 16- and 256-byte aligned, never dereferenced
+
+
+def _ws_args(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=None, offs=None, B=1, S=256, Hq=8, Hkv=2, D=128, table=T16,
+             rows=256, kc=None, vc=None, Lmax=0, ws=T16, ws_bytes=1 << 40)
+    a.update(kw)
+    return tuple(a.values())
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(ws_bytes=256 + 256 * 4 + 256 * 2 * 256 - 1), WORKSPACE),   # one byte short
+    (dict(ws=None), WORKSPACE),
+    (dict(ws=ctypes.c_void_p(4096 + 16)), WORKSPACE),                  # not 256-byte aligned
+    (dict(table=None), INVALID),
+    (dict(rows=255), INVALID),                                        # table shorter than S positions
+    (dict(table=ctypes.c_void_p(4104)), INVALID),                     # table not 16-byte aligned
+    (dict(q=None), INVALID),
+    (dict(Hkv=3), INVALID),
+    (dict(D=64), UNSUPPORTED),
+    (dict(kc=FAKE), INVALID),                                         # one cache without the other
+    (dict(kc=FAKE, vc=FAKE, Lmax=100), INVALID),                      # Lmax < S
+])
+def test_prefill_ws_rejects_before_any_launch(lib, kw, expect):
+    """Every failing check returns before the library touches CUDA (this host
+    has no GPU, so any CUDA call would report LLAMA_ATTN_ERR_CUDA instead)."""
+    assert lib.llama_attn_prefill_ws(*_ws_args(**kw), None) == expect
+
+
+def test_prefill_cp_ws_rejects(lib):
+    f = lib.llama_attn_prefill_cp_ws
+    need = lib.llama_attn_prefill_workspace_size(1, 1024, 2, 128)
+    # q, k, v, out, lse, B, Sq, Skv, Hq, Hkv, D, q_pos_a, q_split, q_pos_b, table, rows, ws, ws_bytes
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 1, 256, 1024, 8, 2, 128, 0, 128, 512, T16, 1024, T16, need - 1,
+             None) == WORKSPACE
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 1, 256, 1024, 8, 2, 128, 0, 128, 512, T16, 1023, T16, need,
+             None) == INVALID  # rows < Skv
+    assert f(FAKE, FAKE, FAKE, FAKE, None, 1, 256, 1024, 8, 2, 128, 64, 128, 512, T16, 1024, T16, need,
+             None) == INVALID  # position not a multiple of 128
+
+
+def test_rope_table_build_rejects(lib):
+    f = lib.llama_attn_rope_table_build
+    need = lib.llama_attn_rope_table_size(1000, 128)
+    assert f(None, need, 1000, 128, 5e5, None) == INVALID
+    assert f(T16, need - 1, 1000, 128, 5e5, None) == WORKSPACE
+    assert f(T16, need, 1000, 128, 0.0, None) == INVALID
+    assert f(T16, need, 0, 128, 5e5, None) == INVALID
+    assert f(ctypes.c_void_p(4100), need, 1000, 128, 5e5, None) == INVALID
+
+
 def test_binding_wraps_every_exported_name():
     for n in la.EXPORTED:
         assert callable(getattr(la, n, None)), f"no Python wrapper named {n}"
