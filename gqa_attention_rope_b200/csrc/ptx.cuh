@@ -316,7 +316,7 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // 2^x evaluated on the FMA pipe (it takes part of the load off the MUFU unit):
 // x = n + f with n = round-to-nearest(x) and f in [-1/2, 1/2]; 2^f by a cubic
 // whose coefficients minimise the maximum relative error on that interval
-// (derived by fit_exp2_poly.py; max relative error 7.5e-5, far below the bf16
+// (derived by tests/fit_exp2_poly.py; max relative error 7.5e-5, far below the bf16
 // rounding of P); 2^n is added to the exponent field. x is clamped at -126 so
 // the exponent stays in range; inputs below that give a result under 2^-125.
 __device__ __forceinline__ float ex2_poly(float x) {

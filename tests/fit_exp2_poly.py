@@ -8,8 +8,8 @@ coefficients minimise the maximum relative error on [-1/2, 1/2]. The
 minimax fit uses Lawson's iteratively reweighted least squares on a dense
 Chebyshev grid (float64).
 
-Run as a script to print the coefficients in the form pasted into
-prefill_bf16.cuh; tests/test_exp2_poly.py re-runs the fit and checks the
+Run as a script to print the coefficients in the form written into
+ex2_poly (gqa_attention_rope_b200/csrc/ptx.cuh); tests/test_exp2_poly.py re-runs the fit and checks the
 kernel's constants and the error bound.
 """
 from __future__ import annotations

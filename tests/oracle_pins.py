@@ -127,6 +127,45 @@ def check_rope_identities(lib):
         assert np.array_equal(yh[:, h], O.rope_rotate(xh[:, h], ph, base, lib=lib))
 
 
+def torch_rope_rotate_half(x, pos, base):
+    """The other common RoPE layout, written out independently: dimension k is
+    paired with dimension k + D/2 (first half, second half) and the pair turns
+    by pos * base^(-2k/D). x [..., T, D] float64, pos [T]."""
+    D = x.shape[-1]
+    inv = base ** (-torch.arange(0, D, 2, dtype=torch.float64) / D)
+    ang = pos[:, None] * inv
+    c, s = torch.cos(ang), torch.sin(ang)
+    x1, x2 = x[..., : D // 2], x[..., D // 2:]
+    return torch.cat([x1 * c - x2 * s, x2 * c + x1 * s], dim=-1)
+
+
+def check_rotate_half_is_a_permutation(lib):
+    """The adjacent-pair rotation (RoFormer's, which the oracle follows) and
+    the rotate-half layout are one method under a fixed permutation of the
+    head dimensions: with P putting the even dimensions first and the odd ones
+    after, rotate_half(P x) = P R(p) x. So attention computed in either layout
+    from correspondingly permuted q and k is the same."""
+    gen = torch.Generator().manual_seed(23)
+    D, base, T = 16, 500000.0, 6
+    perm = torch.cat([torch.arange(0, D, 2), torch.arange(1, D, 2)])
+    x = _rand(gen, T, D)
+    pos = torch.tensor([0.0, 1.0, 5.0, 37.0, 4096.0, 131071.0], dtype=torch.float64)
+    ours = torch.from_numpy(O.rope_rotate(x.numpy(), pos.numpy(), base, lib=lib))
+    half = torch_rope_rotate_half(x[:, perm], pos, base)
+    assert torch.allclose(half, ours[:, perm], rtol=1e-12, atol=1e-12)
+    # attention: the rotate-half layout on permuted q and k = the oracle on the originals
+    B, S, Hq, Hkv = 1, 9, 4, 2
+    q, k, v = _rand(gen, B, S, Hq, D), _rand(gen, B, S, Hkv, D), _rand(gen, B, S, Hkv, D)
+    p = torch.arange(S, dtype=torch.float64)
+    qh = torch_rope_rotate_half(q[..., perm].permute(0, 2, 1, 3), p, base)      # [B, Hq, S, D]
+    kh = torch_rope_rotate_half(k[..., perm].permute(0, 2, 1, 3), p, base)
+    kh = kh.repeat_interleave(Hq // Hkv, dim=1)
+    vh = v.permute(0, 2, 1, 3).repeat_interleave(Hq // Hkv, dim=1)
+    ref = F.scaled_dot_product_attention(qh, kh, vh, is_causal=True).permute(0, 2, 1, 3).numpy()
+    got = O.prefill(q, k, v, None, base, lib=lib)
+    assert np.allclose(got, ref, rtol=1e-10, atol=1e-12)
+
+
 def check_worked_example(lib):
     vals = {}
     with open(os.path.join(GOLDEN, "worked_example_rope_attention.txt")) as f:
@@ -323,6 +362,7 @@ def check_lse(lib):
 ALL_CHECKS = [
     check_rope_freqs_closed_form,
     check_rope_identities,
+    check_rotate_half_is_a_permutation,
     check_worked_example,
     check_bruteforce_vs_torch,
     check_mha_equals_sdpa,

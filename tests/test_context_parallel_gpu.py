@@ -16,6 +16,7 @@ import gqa_attention_rope_b200 as la
 from gqa_attention_rope_b200 import build as labuild
 from gqa_attention_rope_b200 import context_parallel as CP
 from gqa_attention_rope_b200 import workloads as W
+from guards import check_guard, guarded
 from oracle import oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -47,11 +48,16 @@ def test_zigzag_ranks_match_whole_prefill(N, B, S, Hq, Hkv):
     for r in range(N):
         pos_a, pos_b, L = CP.zigzag_chunks(S, N, r)
         q_l = CP.shard_rows(q, N, r)
-        lse_l = torch.full((B, 2 * L, Hq), float("nan"), device="cuda")
-        out_l, _ = la.llama_attn_prefill_cp(q_l, k, v, pos_a, L, pos_b, lse=lse_l)
+        lse_buf, lse_l = guarded((B, 2 * L, Hq), torch.float32)
+        lse_l.fill_(float("nan"))
+        out_buf, out_l = guarded(q_l.shape)
+        la.llama_attn_prefill_cp(q_l, k, v, pos_a, L, pos_b, out=out_l, lse=lse_l)
         outs.append(out_l)
         lses.append(lse_l)
-    torch.cuda.synchronize()
+        bufs = (out_buf, lse_buf)
+        torch.cuda.synchronize()
+        check_guard(bufs[0])
+        check_guard(bufs[1], what="lse")
     got = CP.unshard_rows(outs, N)
     assert torch.equal(got, ref_out), "context-parallel rows differ from the whole-sequence prefill"
     assert torch.equal(CP.unshard_rows(lses, N), ref_lse)
@@ -73,8 +79,10 @@ def test_chunks_match_rows_of_whole_prefill(Skv, pos_a, split, pos_b, Sq):
     rows = np.r_[pos_a:pos_a + split, pos_b:pos_b + (Sq - split)]
     idx = torch.from_numpy(rows).cuda()
     q_l = q[:, idx].contiguous()
-    out_l, _ = la.llama_attn_prefill_cp(q_l, k, v, pos_a, split, pos_b)
+    buf, out_l = guarded(q_l.shape)
+    la.llama_attn_prefill_cp(q_l, k, v, pos_a, split, pos_b, out=out_l)
     torch.cuda.synchronize()
+    check_guard(buf)
     assert torch.equal(out_l, full[:, idx])
     ref = O.prefill(inp["q"], inp["k"], inp["v"], None, w.rope_theta, rows=rows)
     err = np.abs(out_l[0].float().cpu().numpy() - ref).max()

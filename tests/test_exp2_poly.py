@@ -9,7 +9,7 @@ import numpy as np
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 CSRC = os.path.join(ROOT, "gqa_attention_rope_b200", "csrc")
-sys.path.insert(0, CSRC)
+sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
 import fit_exp2_poly as F  # noqa: E402
 
 

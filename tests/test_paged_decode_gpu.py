@@ -16,6 +16,7 @@ import torch
 import gqa_attention_rope_b200 as la
 from gqa_attention_rope_b200 import build as labuild
 from gqa_attention_rope_b200 import workloads as W
+from guards import check_guard, guarded
 from oracle import oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -66,11 +67,13 @@ def test_paged_decode(page_size, lens):
     kp, vp, table = kp.cuda(), vp.cuda(), table.cuda()
     ws_bytes = lib.llama_attn_decode_workspace_size(B, Hq, max_blocks * page_size, 128)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
-    out = torch.empty_like(q)
+    buf, out = guarded(q.shape)
     st = lib.llama_attn_decode_paged(_p(q), _p(kp), _p(vp), _p(table), _p(lens_d), _p(out), B, Hq, Hkv, 128,
                                      page_size, max_blocks, n_pages, ctypes.c_float(w.rope_theta), _p(ws), ws_bytes,
                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0
+    torch.cuda.synchronize()
+    check_guard(buf)
     # the Python binding's wrapper makes the same call
     out_py = la.llama_attn_decode_paged(q, kp, vp, table, lens_d, rope_theta=w.rope_theta)
     ref_gpu = la.llama_attn_decode(q, inp["kcache"].cuda(), inp["vcache"].cuda(), lens_d)

@@ -16,6 +16,7 @@ import torch
 import gqa_attention_rope_b200 as la
 from gqa_attention_rope_b200 import build as labuild
 from gqa_attention_rope_b200 import workloads as W
+from guards import check_guard, guarded
 from oracle import oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -50,10 +51,14 @@ def test_prefill_ex_lse_and_output(B, S, Hq, Hkv, docs):
     inp = W.make_prefill_inputs(w)
     q, k, v = (inp[n].cuda() for n in ("q", "k", "v"))
     offs = inp["doc_offsets"].cuda() if inp["doc_offsets"] is not None else None
-    lse = torch.full((B, S, Hq), float("nan"), dtype=torch.float32, device="cuda")
-    out, _ = la.llama_attn_prefill_ex(q, k, v, lse=lse, doc_offsets=offs)
+    lse_buf, lse = guarded((B, S, Hq), torch.float32)
+    lse.fill_(float("nan"))
+    out_buf, out = guarded(q.shape)
+    la.llama_attn_prefill_ex(q, k, v, out=out, lse=lse, doc_offsets=offs)
     plain = la.llama_attn_prefill(q, k, v, doc_offsets=offs)
     torch.cuda.synchronize()
+    check_guard(out_buf)
+    check_guard(lse_buf, what="lse")
     assert torch.equal(out, plain), "prefill_ex output differs from prefill"
     ref_out, ref_lse = O.prefill_lse(inp["q"], inp["k"], inp["v"], inp["doc_offsets"])
     got_lse = lse.cpu().numpy().astype(np.float64)
@@ -72,10 +77,12 @@ def test_kv_cache_append(docs):
     q, k, v = (inp[n].cuda() for n in ("q", "k", "v"))
     offs = inp["doc_offsets"].cuda() if inp["doc_offsets"] is not None else None
     canary = 7.0
-    kc = torch.full((B, Hkv, Lmax, 128), canary, dtype=torch.bfloat16, device="cuda")
-    vc = torch.full((B, Hkv, Lmax, 128), canary, dtype=torch.bfloat16, device="cuda")
+    kc_buf, kc = guarded((B, Hkv, Lmax, 128), fill=canary)
+    vc_buf, vc = guarded((B, Hkv, Lmax, 128), fill=canary)
     la.llama_attn_prefill_ex(q, k, v, doc_offsets=offs, kcache=kc, vcache=vc)
     torch.cuda.synchronize()
+    check_guard(kc_buf, fill=canary, what="kcache")
+    check_guard(vc_buf, fill=canary, what="vcache")
     kc_h, vc_h = kc.cpu(), vc.cpu()
     # values: copied bit for bit; rows past S untouched
     assert torch.equal(vc_h[:, :, :S], inp["v"].permute(0, 2, 1, 3))

@@ -3,6 +3,8 @@
 document-length ranges, cache-length ranges, the NaN poison past each cached
 sequence, and the unmasked-pair count that the throughput metric divides by
 (checked against a brute-force count of the mask)."""
+import os
+
 import numpy as np
 import torch
 
@@ -68,3 +70,28 @@ def test_unmasked_pairs_matches_mask_count():
                 count += ds[b * w.S + i] == ds[b * w.S + j]  # same document (starts are row-local)
     assert W.unmasked_pairs(inp["doc_offsets"], w.B, w.S) == count
     assert W.unmasked_pairs(None, 3, 10) == 3 * 55
+
+
+def _page_numbers():
+    vals = {}
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "page_shapes.txt")
+    for line in open(path):
+        line = line.split("#")[0].strip()
+        if line:
+            k, v = (x.strip() for x in line.split("="))
+            vals[k] = int(v)
+    return vals
+
+
+def test_workloads_follow_the_pages_head_layouts():
+    """The synthetic workloads carry the head layouts and RoPE base the pages
+    print (tests/golden/page_shapes.txt, each number cited there)."""
+    pg = _page_numbers()
+    for w in (W.PACKED_8B, W.PACKED_405B, W.LONG_128K, W.DECODE_70B):
+        assert w.Hkv == pg["kv_heads_all"], w.name
+        assert w.D * w.Hq // w.Hq == 128 and w.rope_theta == pg["rope_base"], w.name
+    w = W.PACKED_405B
+    assert (w.Hq, w.Hkv) == (pg["heads_405b"], pg["kv_heads_405b"])
+    assert pg["d_model_405b"] // pg["heads_405b"] == w.D  # head_dim = hidden / heads
+    # the long-context base is a value the library accepts as an argument, not the default
+    assert pg["rope_base_long"] == 10 * pg["rope_base"] and pg["rope_base_original"] < pg["rope_base"]

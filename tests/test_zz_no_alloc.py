@@ -1,12 +1,13 @@
 """The allocation-free decode entry point against the regular one.
 
 llama_attn_decode_noalloc serves callers that cannot allocate device memory
-(for example code inside a CUDA graph capture, or under an allocator that owns
-all device memory): its split-KV partials live in a fixed array inside the
-library instead of a caller workspace. This test calls both entry points
-through the C ABI on the same inputs, twice in a row, and requires the
-no-allocation results to match the regular ones within the bf16 tolerance the
-other decode tests use. It sits in its own file, collected last.
+(for example a host whose allocator owns all of device memory): its split-KV
+partials live in a fixed array inside the library instead of a caller
+workspace. This test calls both entry points through the C ABI on the same
+inputs, twice in a row, and requires the no-allocation results to match the
+regular ones within the bf16 tolerance the other decode tests use; the second
+call must leave the device's free memory unchanged. It sits in its own file,
+collected last.
 """
 import ctypes
 
@@ -45,12 +46,16 @@ def test_noalloc_decode_matches_regular_decode_twice():
         st = lib.llama_attn_decode(_p(q), _p(kc), _p(vc), _p(ln), _p(ref), w.B, w.Hq, w.Hkv, w.D, w.Lmax,
                                    ctypes.c_float(w.rope_theta), _p(ws), ws_bytes, stream)
         assert st == 0
-        for _ in range(2):
-            out = torch.full_like(q, float("nan"))
+        outs = [torch.full_like(q, float("nan")) for _ in range(2)]
+        torch.cuda.synchronize()
+        for i, out in enumerate(outs):
+            free0 = torch.cuda.mem_get_info()[0]
             st = lib.llama_attn_decode_noalloc(_p(q), _p(kc), _p(vc), _p(ln), _p(out), w.B, w.Hq, w.Hkv, w.D,
                                                w.Lmax, ctypes.c_float(w.rope_theta), stream)
             assert st == 0
             torch.cuda.synchronize()
+            if i > 0:  # the first call on a device may still load the kernels
+                assert torch.cuda.mem_get_info()[0] == free0, "the no-alloc decode changed device free memory"
             assert torch.isfinite(out.float()).all()
             err = (out.float() - ref.float()).abs().max().item()
             assert err <= TOL_BF16, f"no-alloc decode differs from decode by {err}"
