@@ -1,22 +1,27 @@
 """Benchmark of the attention hot path on B200.
 
-Default workload (one GPU): the 8B-shaped packed prefill, B=4, S=8192, Hq=32,
-Hkv=8, D=128, bf16, causal + cross-document mask with documents U[512, 4096].
-One step is one llama_attn_prefill call over that batch (document layout,
-K rotation, tensor-core attention). The metric counts only unmasked (i, j)
-pairs: FLOPs = 4 * D * Hq * pairs. The decode form of the hot path (70B-shaped,
-64 sequences, Hq=64, Hkv=8, cache lengths U[1024, 32768]) is measured in the
-same run after the timed prefill steps and reported under "decode" (GB/s of
-cached K/V rows read).
+Headline workload (one GPU): the 128K long-context prefill, B=1, S=131072,
+Hq=32, Hkv=8, D=128, bf16, one causal document (the largest single-GPU
+workload). One step is one llama_attn_prefill call over that batch (K
+rotation, tensor-core attention). The metric counts only unmasked (i, j)
+pairs: FLOPs = 4 * D * Hq * pairs. In the same run the other prefill
+workloads (8B-shaped packed, B=4, S=8192, Hq=32, documents U[512, 4096];
+405B-shaped, B=1, S=16384, Hq=128, documents U[1024, 8192]) are timed the same
+way and reported under "prefill_workloads", each with its own roofline, end to
+end figure and CPU baseline; the decode form (70B-shaped, 64 sequences, Hq=64,
+Hkv=8, cache lengths U[1024, 32768]) is reported under "decode" (GB/s of cached
+K/V rows read).
 
 `--impl reference` times the float64 CPU oracle on the host cores instead, on
 a bounded sample of query rows of the same workload, in the same unit.
 
-Multi-GPU (torchrun): one process per GPU, each with its own independent
-batch (weak scaling, no data-path collective); rank 0 prints the line, value =
-FLOPs of all ranks / max-over-ranks time.
+Multi-GPU (torchrun): by default one process per GPU, each with its own
+independent batch (weak scaling, no data-path collective); rank 0 prints the
+line, value = FLOPs of all ranks / max-over-ranks time.
 
 Options that add measurements of the paths around the hot path:
+  --shard kv-groups  one workload split over the GPUs by KV group (each rank
+                     its Hkv/N KV heads and their query heads; strong scaling)
   --cp               context-parallel prefill of one single-document workload
                      over the GPUs (zigzag split, K/V all-gather, strong scaling)
   --prefill-ex       the prefill with its LSE output and KV-cache append
@@ -45,18 +50,27 @@ L2_FLUSH_BYTES = 256 << 20
 
 
 def load_peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, "measured" or
+    "fallback"): the measured copy bandwidth and cuBLAS bf16 throughput of this
+    pool's B200s, else the earlier pool measurement."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             pk = json.load(f)
-        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained", 0)), "measured"
+        burst = float(pk["bf16_tflops"])
+        return float(pk["hbm_gbs"]), burst, float(pk.get("bf16_tflops_sustained") or burst), "measured"
     except Exception:
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+# A kernel timed for longer than this in one timed region runs at the power
+# cap's sustained clock, so it is compared with the sustained tensor peak.
+SUSTAINED_AFTER_S = 1.0
+
+
 class ClockSampler:
-    """SM clock and clock-event reasons sampled every 5 ms (NVML, in a thread)
-    while the timed region runs; falls back to nvidia-smi."""
+    """SM clock and clock-event reasons sampled every 5 ms through NVML (in a
+    thread) while the timed region runs; without NVML the record says so."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
@@ -207,32 +221,52 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
-def config_of(w, world):
+def config_of(w, world, shard="replicas"):
+    if world == 1:
+        par = "1 GPU"
+    elif shard == "kv-groups":
+        par = f"one workload split by KV group over {world} GPUs ({w.Hkv // world} KV heads per GPU; strong scaling)"
+    else:
+        par = f"{world} independent replicas (weak scaling)"
     return {"workload": w.name, "B": w.B, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
             "doc_lengths": None if w.doc_range is None else f"U[{w.doc_range[0]},{w.doc_range[1]}]",
             "rope_theta": w.rope_theta, "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)",
-            "parallelism": f"{world} independent replicas (weak scaling)" if world > 1 else "1 GPU"}
+            "parallelism": par}
 
 
 # ---------------------------------------------------------------- GPU arm
 
-def run_ours(args, w):
-    import gqa_attention_rope_b200 as la
-    world, rank, local = dist_setup(args.gpus)
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    la.lib()
-    hbm_peak, tc_peak, tc_sust, peak_kind = load_peaks()
+def cpu_baseline_of(w, inp, seconds):
+    f, s, n, threads = oracle_rows_sample(w, inp, seconds)
+    return {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{n} random query rows x {w.Hq} heads of {w.name} (float64 C oracle, "
+                      f"full masked rows, {s:.1f} s)"}
 
-    # inputs: per-rank seed so ranks hold independent batches
-    wr = W.PrefillWorkload(w.name, w.seed + 1000 * rank, w.B, w.S, w.Hq, w.Hkv, w.D, w.dtype, w.doc_range,
-                           w.rope_theta)
-    inp = W.make_prefill_inputs(wr)
+
+def measure_prefill(args, la, dev, w, world, rank, peaks, cpu_seconds, steps):
+    """Times `steps` prefill steps of workload w on this rank (device time,
+    CUDA events, L2 flushed between steps), then the same steps end to end
+    through the public API with pinned host buffers. Returns one record."""
+    hbm_peak, tc_peak, tc_sust, peak_kind = peaks
+    shard = args.shard if world > 1 else "replicas"
+    if shard == "kv-groups":
+        # the same workload on every rank; this rank's KV groups and their query heads
+        from gqa_attention_rope_b200 import kv_group_parallel as KG
+        full = W.make_prefill_inputs(w)
+        q_h, k_h, v_h = KG.shard_qkv(full["q"], full["k"], full["v"], world, rank)
+        inp = dict(q=q_h, k=k_h, v=v_h, doc_offsets=full["doc_offsets"])
+        wr = w
+        heads_local = q_h.shape[2]
+    else:
+        wr = W.PrefillWorkload(w.name, w.seed + 1000 * rank, w.B, w.S, w.Hq, w.Hkv, w.D, w.dtype, w.doc_range,
+                               w.rope_theta)  # per-rank seed: ranks hold independent batches
+        inp = W.make_prefill_inputs(wr)
+        heads_local = w.Hq
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
     offs = inp["doc_offsets"].to(dev) if inp["doc_offsets"] is not None else None
     out = torch.empty_like(q)
     pairs = W.unmasked_pairs(inp["doc_offsets"], wr.B, wr.S)
-    flops = 4.0 * w.D * w.Hq * pairs
+    flops = 4.0 * w.D * heads_local * pairs  # this rank's FLOPs per step
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -245,13 +279,13 @@ def run_ours(args, w):
     if la.llama_attn_get_device_error() != 0:
         raise RuntimeError("device error word set during warm-up")
 
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev.index)
     clocks.start()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize()
     la.llama_attn_profile_begin()
-    for i in range(args.steps):
+    for i in range(steps):
         flush.zero_()
         ev[i][0].record(stream)
         step()
@@ -262,10 +296,12 @@ def run_ours(args, w):
     clk = clocks.stop()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = max_over_ranks(sum(step_ms), world)
-    all_flops = sum_over_ranks(flops * args.steps, world)
+    all_flops = sum_over_ranks(flops * steps, world)
     value = all_flops / (total_ms / 1e3) / 1e12
     kernel_ms = main_ms / max(main_n, 1)
     achieved = flops / (kernel_ms / 1e3) / 1e12
+    sustained = kernel_ms * steps / 1e3 > SUSTAINED_AFTER_S
+    peak = tc_sust if sustained else tc_peak
 
     # end to end through the public API: pinned host inputs -> device -> call -> host result
     hq, hk, hv = (inp[n].pin_memory() for n in ("q", "k", "v"))
@@ -286,9 +322,9 @@ def run_ours(args, w):
     for _ in range(2):
         e2e_step()
     torch.cuda.synchronize()
-    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier(world)
-    for i in range(args.steps):
+    for i in range(steps):
         e_ev[i][0].record(stream)
         e2e_step()
         e_ev[i][1].record(stream)
@@ -298,35 +334,71 @@ def run_ours(args, w):
     d2h = hout.numel() * hout.element_size()
     e2e = {"value": all_flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h}
-    del hq, hk, hv, hout, dq, dk, dv, dout
+    if la.llama_attn_get_device_error() != 0:
+        raise RuntimeError("device error word set during the benchmark")
+    cpu = None
+    if rank == 0 and world == 1 and cpu_seconds > 0:
+        cpu = cpu_baseline_of(wr, inp, cpu_seconds)
+    return {
+        "workload": w.name, "value": value, "unit": "TFLOP/s", "steps": steps, "ms_per_step": total_ms / steps,
+        "flops_per_step_per_gpu": flops, "unmasked_pairs_per_head": pairs,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak,
+                     "peak_kind": f"{peak_kind} bf16 dense ({'sustained' if sustained else 'burst'})",
+                     "kernel": "prefill_bf16_kernel", "kernel_ms": kernel_ms,
+                     "traffic": load_traffic("prefill_bf16_kernel", w.name)},
+        "cpu_baseline": cpu, "e2e": e2e, "clocks": clk, "gpu_launches": launches,
+        "config": config_of(w, world, shard),
+    }
 
+
+def run_ours(args, w):
+    import gqa_attention_rope_b200 as la
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    la.lib()
+    peaks = load_peaks()
+    if args.shard == "kv-groups" and w.Hkv % world != 0:
+        raise SystemExit(f"--shard kv-groups needs the GPU count to divide Hkv = {w.Hkv}")
+
+    head = measure_prefill(args, la, dev, w, world, rank, peaks, 0 if args.no_cpu_baseline else args.cpu_seconds,
+                           args.steps)
+    extras = {}
+    for name in ([] if args.no_extra else [n for n in args.extra_workloads.split(",") if n and n != w.name]):
+        wx = W.WORKLOADS[name]
+        if args.shard == "kv-groups" and wx.Hkv % world != 0:
+            continue
+        rec = measure_prefill(args, la, dev, wx, world, rank, peaks,
+                              0 if args.no_cpu_baseline else args.extra_cpu_seconds, max(args.steps, 10))
+        extras[name] = rec
+    hbm_peak, tc_peak, tc_sust, peak_kind = peaks
     decode = None if args.no_decode else run_decode(args, la, dev, world, rank, hbm_peak, peak_kind)
+    wr = W.PrefillWorkload(w.name, w.seed + 1000 * rank, w.B, w.S, w.Hq, w.Hkv, w.D, w.dtype, w.doc_range,
+                           w.rope_theta)
     qkv = run_qkv_fp8(args, la, dev, wr, tc_peak, peak_kind) if args.qkv_fp8 else None
-    pex = run_prefill_ex(args, la, dev, wr, q, k, v, offs, flops, tc_peak, peak_kind) if args.prefill_ex else None
+    pex = run_prefill_ex(args, la, dev, wr, tc_peak, peak_kind) if args.prefill_ex else None
     if la.llama_attn_get_device_error() != 0:
         raise RuntimeError("device error word set during the benchmark")
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        f, s, n, threads = oracle_rows_sample(wr, inp, args.cpu_seconds)
-        cpu = {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-               "sample": f"{n} random query rows x {w.Hq} heads of {w.name} (float64 C oracle, "
-                         f"full masked rows, {s:.1f} s)"}
-
-    traffic = load_traffic("prefill_bf16_kernel", w.name)
     line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
-        "warmup": max(3, args.warmup), "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(config_of(w, world), flops_per_step_per_gpu=flops, unmasked_pairs_per_head=pairs),
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                     "frac": achieved / tc_peak, "peak_kind": f"{peak_kind} bf16 dense (burst)",
-                     "kernel": "prefill_bf16_kernel", "kernel_ms": kernel_ms, "traffic": traffic},
-        "cpu_baseline": cpu,
-        "e2e": e2e,
-        "clocks": clk,
-        "gpu_launches": (launches + (decode["gpu_launches"] if decode else 0) + (qkv["gpu_launches"] if qkv else 0)
+        "metric": METRIC, "value": head["value"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "strong" if (world > 1 and args.shard == "kv-groups") else "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(head["config"], flops_per_step_per_gpu=head["flops_per_step_per_gpu"],
+                       unmasked_pairs_per_head=head["unmasked_pairs_per_head"]),
+        "roofline": head["roofline"],
+        "cpu_baseline": head["cpu_baseline"],
+        "e2e": head["e2e"],
+        "clocks": head["clocks"],
+        "gpu_launches": (head["gpu_launches"] + sum(r["gpu_launches"] for r in extras.values())
+                         + (decode["gpu_launches"] if decode else 0) + (qkv["gpu_launches"] if qkv else 0)
                          + (pex["gpu_launches"] if pex else 0)),
+        "prefill_workloads": {n: {k: r[k] for k in ("value", "unit", "steps", "ms_per_step",
+                                                    "flops_per_step_per_gpu", "unmasked_pairs_per_head", "roofline",
+                                                    "e2e", "cpu_baseline", "clocks", "gpu_launches", "config")}
+                              for n, r in extras.items()},
         "decode": decode,
     }
     if qkv is not None:
@@ -393,6 +465,8 @@ def run_cp(args, w):
     value = flops_total * args.steps / (total_ms / 1e3) / 1e12
     kernel_ms = main_ms / max(main_n, 1)
     achieved = flops_local / (kernel_ms / 1e3) / 1e12
+    sustained = kernel_ms * args.steps / 1e3 > SUSTAINED_AFTER_S
+    peak = tc_sust if sustained else tc_peak
 
     # end to end: the rank's pinned host shards in, its output rows back
     hq, hk, hv = (t.cpu().pin_memory() for t in (ql, kl, vl))
@@ -433,8 +507,9 @@ def run_cp(args, w):
         "warmup": max(3, args.warmup), "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(cfg, flops_per_step_total=flops_total),
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s",
-                     "frac": achieved / tc_peak, "peak_kind": f"{peak_kind} bf16 dense (burst)",
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak,
+                     "peak_kind": f"{peak_kind} bf16 dense ({'sustained' if sustained else 'burst'})",
                      "kernel": "prefill_bf16_kernel", "kernel_ms": kernel_ms, "traffic": None},
         "cpu_baseline": cpu,
         "e2e": {"value": flops_total * args.steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
@@ -450,9 +525,13 @@ def run_cp(args, w):
         dist.destroy_process_group()
 
 
-def run_prefill_ex(args, la, dev, w, q, k, v, offs, flops, tc_peak, peak_kind):
+def run_prefill_ex(args, la, dev, w, tc_peak, peak_kind):
     """The prefill step with its two decode-linking outputs: per-row LSE and the
     append of rotated K and V to a [B, Hkv, S, D] decode-layout cache."""
+    inp = W.make_prefill_inputs(w)
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    offs = inp["doc_offsets"].to(dev) if inp["doc_offsets"] is not None else None
+    flops = 4.0 * w.D * w.Hq * W.unmasked_pairs(inp["doc_offsets"], w.B, w.S)
     out = torch.empty_like(q)
     lse = torch.empty(w.B, w.S, w.Hq, dtype=torch.float32, device=dev)
     kc = torch.empty(w.B, w.Hkv, w.S, w.D, dtype=torch.bfloat16, device=dev)
@@ -646,11 +725,18 @@ def load_traffic(kernel: str, workload: str):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=W.PACKED_8B.name, choices=[n for n, x in W.WORKLOADS.items()
-                                                                      if isinstance(x, W.PrefillWorkload)])
+    prefill_names = [n for n, x in W.WORKLOADS.items() if isinstance(x, W.PrefillWorkload) and x.dtype == "bf16"]
+    ap.add_argument("--workload", default=W.LONG_128K.name, choices=prefill_names,
+                    help="the headline prefill workload (the line's value)")
+    ap.add_argument("--extra-workloads", default=",".join([W.PACKED_8B.name, W.PACKED_405B.name]),
+                    help="comma-separated prefill workloads also timed and reported under prefill_workloads")
+    ap.add_argument("--no-extra", action="store_true", help="time the headline workload only")
+    ap.add_argument("--extra-cpu-seconds", type=float, default=8.0)
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "kv-groups"],
+                    help="N>1: independent replicas per GPU (weak), or one workload split by KV group (strong)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-seqs", type=int, default=W.DECODE_70B.B,
                     help="sequences in the decode batch (64 = the 70B-shaped workload)")
