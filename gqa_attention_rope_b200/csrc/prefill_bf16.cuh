@@ -4,8 +4,11 @@
 // One CTA computes a 128-row query tile for NH (1 or 2) query heads of the same
 // KV group, so every K/V tile brought in by TMA serves both heads (GQA reuse).
 //
-//   warp 0      TMA producer: Q tiles once, then K/V tiles through a 3-stage ring
-//               in the order the MMA warp consumes them (K0, K1, V0, K2, V1, ...).
+//   warp 0      TMA producer: Q tiles once per item, then K tiles through a
+//               2-stage K ring and V tiles through a 1-stage V ring, issued in
+//               the order K0, K1, V0, K2, V1, ..., so each K tile is loaded
+//               one tile ahead of its S MMAs and each V tile while the softmax
+//               of its tile runs.
 //   warp 1      TMEM owner; one thread issues S_h = Q_h K_j^T (M=128, N=128,
 //               K=128; fp32 accumulators in TMEM)
 //   warp 2      one thread issues O_h += P_h V_j (P from shared memory, V MN-major).
@@ -14,6 +17,8 @@
 //               has completed) would otherwise leave the tensor pipe idle; with
 //               S and PV issued from different threads one thread's waits
 //               overlap the other's MMAs.
+//   Registers: the four role warps (one warpgroup) hold 64 each and give the
+//   rest to the eight softmax warps, which hold 216 each (setmaxnreg).
 //   warps 4-7   softmax for head slot 0, warps 8-11 for slot 1: thread = query
 //               row = TMEM lane. Rotates its Q row in shared memory (RoPE at the
 //               row's document position), then per KV tile: S from TMEM ->
@@ -23,8 +28,8 @@
 //               same reference max); epilogue O/l -> bf16 -> TMA store.
 //
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
-// Shared memory (1024-aligned): Q_0, Q_1 (32 KB each), K/V ring 3 x 32 KB,
-// P_0, P_1 (32 KB each), barriers. Every 32 KB tile is two 64-column halves of
+// Shared memory (1024-aligned): Q_0, Q_1 (32 KB each), K ring 2 x 32 KB, V ring
+// 32 KB, P_0, P_1 (32 KB each), barriers. Every 32 KB tile is two 64-column halves of
 // 128 rows x 128 B in the 128B-swizzled layout TMA writes.
 //
 // KV tiles run from the tile holding the document start of the first query
@@ -45,7 +50,7 @@ namespace pfx {
 
 constexpr int BM = 128;
 constexpr int BN = 128;
-constexpr int NSTAGE = 3;
+constexpr int NSTAGE = 3;  // 32 KB ring stages, K and V rings together
 constexpr uint32_t TILE = 32768;
 constexpr uint32_t HALF = 16384;
 constexpr uint32_t OFF_Q = 0;
@@ -58,15 +63,21 @@ constexpr int NTHREADS = 384;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float kRescaleLog2 = 8.0f;
 
-// Each ring stage has one full barrier per tile kind: a K tile landing in a
-// stage completes a phase of that stage's K_FULL barrier, a V tile one of its
-// V_FULL barrier. Each issuer waits only on its own kind, in consecutive
-// phases, so no wait depends on the order in which separate TMA loads land.
+// K tiles go through a ring of NK stages and V tiles through a ring of NV
+// stages (in that order in the ring area); each stage has a full barrier (the
+// TMA load's bytes landed) and an empty barrier (the MMAs that read it
+// completed). The S issuer waits only on the K ring's full barriers and the PV
+// issuer only on the V ring's, each in consecutive phases (tile count /
+// stages), so a wait can neither alias nor pass early whatever order separate
+// TMA loads land in. Of the splits of the three 32 KB stages, two K stages and
+// one V stage measured best: a V tile is needed a whole softmax after its K.
+constexpr int NK = 2, NV = 1;
 enum : int {
   B_K_FULL = 0,
-  B_V_FULL = B_K_FULL + NSTAGE,
-  B_KV_EMPTY = B_V_FULL + NSTAGE,
-  B_Q_FULL = B_KV_EMPTY + NSTAGE,
+  B_K_EMPTY = B_K_FULL + NK,
+  B_V_FULL = B_K_EMPTY + NK,
+  B_V_EMPTY = B_V_FULL + NV,
+  B_Q_FULL = B_V_EMPTY + NV,
   B_Q_READY,
   B_S_READY = B_Q_READY + 2,
   B_S_FREE = B_S_READY + 2,
@@ -139,7 +150,7 @@ __device__ __forceinline__ Item item_of(int item, const Params& p) {
 // The producer publishes each claimed item id in an 8-entry shared-memory ring
 // as soon as it is claimed (well before its Q tiles are loaded); -1 ends every
 // role's loop.
-// The K/V ring index and the per-tile barrier phases run on across items; the
+// The ring counters and the per-tile barrier phases run on across items; the
 // next item's Q tiles are loaded as soon as the S MMAs of the current item have
 // finished reading Q, and the output tile is staged in the P buffer and stored
 // by warp 3, so one item's tail overlaps the next item's start.
@@ -163,10 +174,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int n_items = p.B * p.n_qt * p.n_hp;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < NSTAGE; ++s) {
+    for (int s = 0; s < NK; ++s) {
       mbar_init(bar(B_K_FULL + s), 1);
+      mbar_init(bar(B_K_EMPTY + s), 1);
+    }
+    for (int s = 0; s < NV; ++s) {
       mbar_init(bar(B_V_FULL + s), 1);
-      mbar_init(bar(B_KV_EMPTY + s), 1);
+      mbar_init(bar(B_V_EMPTY + s), 1);
     }
     mbar_init(bar(B_Q_FULL), 1);
     mbar_init(bar(B_Q_FREE), 2);  // the S issuer's commit and the PV issuer's arrival
@@ -200,457 +214,456 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      uint32_t idx = 0;  // running ring index
-      // Per stage and tile kind: bit st of *_any says a load of that kind went
-      // into stage st, bit st of *_par is the parity of their count.
-      uint32_t k_any = 0, k_par = 0, v_any = 0, v_par = 0;
-      bool ok = true;
-      auto load = [&](bool is_v, int g, int kv_row, int b) -> bool {
-        const uint32_t st = idx % NSTAGE, use = idx / NSTAGE;
-        if (use > 0 && !mbar_wait_backoff(bar(B_KV_EMPTY + st), (use - 1) & 1, wc)) return false;
-        const uint32_t full = bar((is_v ? B_V_FULL : B_K_FULL) + static_cast<int>(st));
-        const CUtensorMap* tm = is_v ? &tm_v : &tm_k;
-        mbar_arrive_expect_tx(full, TILE);
-        tma_load_4d(sbase + OFF_KV + st * TILE, tm, full, 0, g, kv_row, b);
-        tma_load_4d(sbase + OFF_KV + st * TILE + HALF, tm, full, 64, g, kv_row, b);
-        if (is_v) {
-          v_any |= 1u << st;
-          v_par ^= 1u << st;
-        } else {
-          k_any |= 1u << st;
-          k_par ^= 1u << st;
+  // Registers: the role warpgroup (warps 0-3) gives up registers to the two
+  // softmax warpgroups: 64 * 128 + 2 * 216 * 128 = 63,488, within the launch's
+  // 384 threads x 168 = 64,512. Each setmaxnreg heads its warpgroup's branch, so the
+  // compiler allocates every role's code for the count that warpgroup holds.
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 64;");
+    if (warp == 0) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        uint32_t kt = 0, vt = 0;  // K and V tiles loaded so far
+        bool ok = true;
+        // One tile into stage (count % n) of its ring, after the stage's previous
+        // tile has been consumed (empty barrier, phase count / n - 1).
+        auto load_tile = [&](const CUtensorMap* tm, uint32_t& count, int n, int b_full, int b_empty, uint32_t off,
+                             int g, int kv_row, int b) -> bool {
+          const uint32_t st = count % n, use = count / n;
+          if (use > 0 && !mbar_wait_backoff(bar(b_empty + st), (use - 1) & 1, wc)) return false;
+          const uint32_t full = bar(b_full + static_cast<int>(st));
+          mbar_arrive_expect_tx(full, TILE);
+          tma_load_4d(sbase + off + st * TILE, tm, full, 0, g, kv_row, b);
+          tma_load_4d(sbase + off + st * TILE + HALF, tm, full, 64, g, kv_row, b);
+          ++count;
+          return true;
+        };
+        auto load_k = [&](int g, int kv_row, int b) {
+          return load_tile(&tm_k, kt, NK, B_K_FULL, B_K_EMPTY, OFF_KV, g, kv_row, b);
+        };
+        auto load_v = [&](int g, int kv_row, int b) {
+          return load_tile(&tm_v, vt, NV, B_V_FULL, B_V_EMPTY, OFF_KV + NK * TILE, g, kv_row, b);
+        };
+        // The RoPE table rows an item's Q rotation will read: positions
+        // q0 - ds(q0) .. +127 and, when a document starts inside the tile, 0 .. 127.
+        auto prefetch_rows = [&](int v) {
+          if (v < 0 || v >= n_items || p.q_rotated) return;
+          const Item J = item_of(v, p);
+          const int ds0 = p.doc_start ? p.doc_start[J.rowbase + J.q0] : 0;
+          const int p0 = q_global(J.q0, p) - ds0;
+          const int n0 = min(BM, p.n_pos - p0);
+          if (n0 > 0) bulk_prefetch_l2(p.rope_tab + static_cast<int64_t>(p0) * 32, static_cast<uint32_t>(n0) * 512u);
+          if (J.ds_last > J.q0) bulk_prefetch_l2(p.rope_tab, static_cast<uint32_t>(min(BM, p.n_pos)) * 512u);
+        };
+        auto publish = [&](int k, int v) {
+          ring_item[k % kItemRing] = v;
+          __threadfence_block();
+          ring_seq[k % kItemRing] = k;
+        };
+        int it = 0, item = blockIdx.x;
+        int next_item = (item < n_items) ? atomicAdd(p.sched, 1) + static_cast<int>(gridDim.x) : n_items;
+        bool ended = false;
+        publish(0, item < n_items ? item : -1);
+        prefetch_rows(item);
+        for (;; ++it) {
+          if (it > 0 && !mbar_wait_backoff(bar(B_Q_FREE), (it - 1) & 1, wc)) {
+            ok = false;
+            break;
+          }
+          if (item >= n_items) {
+            mbar_arrive(bar(B_Q_FULL));
+            ended = true;
+            break;
+          }
+          const Item I = item_of(item, p);
+          mbar_arrive_expect_tx(bar(B_Q_FULL), static_cast<uint32_t>(p.NH) * TILE);
+          for (int s = 0; s < p.NH; ++s)
+            for (int hf = 0; hf < 2; ++hf)
+              tma_load_4d(sbase + OFF_Q + s * TILE + hf * HALF, &tm_q, bar(B_Q_FULL), hf * 64, I.h0 + s, I.q0, I.b);
+          item = next_item;
+          next_item = (item < n_items) ? atomicAdd(p.sched, 1) + static_cast<int>(gridDim.x) : n_items;
+          publish(it + 1, item < n_items ? item : -1);
+          prefetch_rows(item);
+          ok = load_k(I.g, I.kv_t0 * BN, I.b);
+          for (int j = 1; ok && j < I.n_kv; ++j)
+            ok = load_k(I.g, (I.kv_t0 + j) * BN, I.b) && load_v(I.g, (I.kv_t0 + j - 1) * BN, I.b);
+          if (ok) ok = load_v(I.g, (I.kv_t0 + I.n_kv - 1) * BN, I.b);
+          if (!ok) {
+            ++it;
+            break;
+          }
         }
-        ++idx;
+        // Every issued load has landed before this CTA may exit (these return at
+        // once in the normal flow, where every load was consumed).
+        if (!ended && it > 0) mbar_wait(bar(B_Q_FULL), (it - 1) & 1, wc);
+        // Only the last tile into a stage can still be in flight (each load
+        // waited for the stage to be emptied): wait for the latest phase of each.
+        for (uint32_t st = 0; st < NK; ++st)
+          if (kt > st) mbar_wait(bar(B_K_FULL + static_cast<int>(st)), ((kt - 1 - st) / NK) & 1, wc);
+        for (uint32_t st = 0; st < NV; ++st)
+          if (vt > st) mbar_wait(bar(B_V_FULL + static_cast<int>(st)), ((vt - 1 - st) / NV) & 1, wc);
+      }
+    } else if (warp == 1 || warp == 2) {
+      // ------------------------------------------------------------ MMA issuers
+      // Tile T (counted over all items) sits in K stage T % NK and V stage
+      // T % NV, loaded there for the (T / NK)-th and (T / NV)-th time.
+      if (lane == 0) {
+        constexpr uint32_t idesc_qk = umma_idesc_bf16_f32(128, 128, 0);
+        constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 128, 1);
+        bool ok = true;
+        uint32_t tiles = 0;
+
+        for (int it = 0; ok; ++it) {
+          if (!mbar_wait(bar(B_Q_FULL), it & 1, wc)) break;
+          // The PV issuer waits on Q_FULL only to learn the item id; its arrival
+          // on Q_FREE keeps the next Q load behind this wait, so its parity wait
+          // can never fall two phases behind.
+          if (warp == 2) mbar_arrive(bar(B_Q_FREE));
+          const int item = ring_item[it % kItemRing];
+          if (item < 0 || item >= n_items) break;
+          const Item I = item_of(item, p);
+          if (warp == 1) {
+            for (int s = 0; s < p.NH; ++s) ok = ok && mbar_wait(bar(B_Q_READY + s), it & 1, wc);
+            for (int j = 0; ok && j < I.n_kv; ++j) {
+              const uint32_t T = tiles + j;  // K tile count = tile count
+              const uint32_t st = T % NK;
+              if (!mbar_wait(bar(B_K_FULL + static_cast<int>(st)), (T / NK) & 1, wc)) {
+                ok = false;
+                break;
+              }
+              const uint64_t db = kdesc(sbase + OFF_KV + st * TILE);
+              for (int s = 0; s < p.NH; ++s) {
+                if (T > 0 && !mbar_wait(bar(B_S_FREE + s), (T - 1) & 1, wc)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+                const uint64_t da = kdesc(sbase + OFF_Q + s * TILE);
+  #pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                  const uint64_t off = ((kk >> 2) * HALF + (kk & 3) * 32) >> 4;
+                  tc_mma_ss(tmem + s * 128, da + off, db + off, idesc_qk, kk > 0);
+                }
+                tc_commit(bar(B_S_READY + s));
+              }
+              tc_commit(bar(B_K_EMPTY + static_cast<int>(st)));
+            }
+            tc_commit(bar(B_Q_FREE));  // the Q tiles are free once these MMAs complete
+          } else {
+            for (int j = 0; ok && j < I.n_kv; ++j) {
+              const uint32_t T = tiles + j;  // V tile count = tile count
+              const uint32_t st = T % NV;
+              if (!mbar_wait(bar(B_V_FULL + static_cast<int>(st)), (T / NV) & 1, wc)) {
+                ok = false;
+                break;
+              }
+              const uint64_t db = vdesc(sbase + OFF_KV + (NK + st) * TILE);
+              for (int s = 0; s < p.NH; ++s) {
+                if (!mbar_wait(bar(B_P_READY + s), T & 1, wc)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+                const uint64_t da = kdesc(sbase + OFF_P + s * TILE);
+  #pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                  const uint64_t aoff = ((kk >> 2) * HALF + (kk & 3) * 32) >> 4;
+                  tc_mma_ss(tmem + 256 + s * 128, da + aoff, db + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                            (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(bar(B_PV_DONE + s));
+              }
+              tc_commit(bar(B_V_EMPTY + static_cast<int>(st)));
+            }
+          }
+          tiles += static_cast<uint32_t>(I.n_kv);
+        }
+        // all issued MMAs complete before TMEM may be freed
+        const int drain = (warp == 1) ? B_DRAIN : B_DRAIN_PV;
+        tc_commit(bar(drain));
+        mbar_wait(bar(drain), 0, wc);
+      }
+    } else if (warp == 3) {
+      // ------------------------------------------------------------ output stores
+      if (lane == 0) {
+        bool ok = true;
+        for (int it = 0; ok; ++it) {
+          if (!mbar_wait_backoff(bar(B_O_STAGED + 0), it & 1, wc)) break;
+          const int item = ring_item[it % kItemRing];
+          if (item < 0 || item >= n_items) break;
+          const Item I = item_of(item, p);
+          for (int s = 0; ok && s < p.NH; ++s) {
+            if (s > 0 && !mbar_wait_backoff(bar(B_O_STAGED + s), it & 1, wc)) {
+              ok = false;
+              break;
+            }
+            tma_store_4d(&tm_o, sbase + OFF_P + s * TILE, 0, I.h0 + s, I.q0, I.b);
+            tma_store_4d(&tm_o, sbase + OFF_P + s * TILE + HALF, 64, I.h0 + s, I.q0, I.b);
+            tma_store_commit();
+            tma_store_wait_read0();  // the P buffer may be rewritten from here on
+            mbar_arrive(bar(B_O_READ + s));
+          }
+        }
+        tma_store_wait0();
+      }
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 216;");
+    if ((warp - 4) / 4 < p.NH) {
+      // ------------------------------------------------------------ softmax
+      const int s = (warp - 4) >> 2;
+      const int wq = warp & 3;
+      const int r = wq * 32 + lane;
+      const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+      const uint32_t tS = tmem + lane_off + s * 128;
+      const uint32_t tO = tmem + lane_off + 256 + s * 128;
+      uint8_t* qtile = smem + OFF_Q + s * TILE;
+      uint8_t* ptile = smem + OFF_P + s * TILE;
+      const float sl2 = p.scale_log2;
+      bool ok = true;
+      uint32_t tiles = 0;
+      Item I;
+      int qi_c = 0, ds_i = 0;  // global position of this thread's (clamped) row; its document start
+      // Starts item `it`: reads its id from the ring, loads its row data, waits for
+      // its Q tile and rotates this thread's row in place. False at the end of the
+      // items (or on a timeout, which also clears ok).
+      auto begin_item = [&](int it) -> bool {
+        int item = -1;
+        {
+          const unsigned long long t0 = global_ns();
+          for (uint32_t k = 0;; ++k) {
+            if (ring_seq[it % kItemRing] == it) {
+              __threadfence_block();  // the item id was written before its sequence number
+              item = ring_item[it % kItemRing];
+              break;
+            }
+            if ((k & 63u) == 63u && (wc.aborted() || global_ns() - t0 > kWaitTimeoutNs)) {
+              if (!wc.aborted()) {
+                raise_error(LLAMA_ATTN_DEVERR_TIMEOUT);
+                atomicExch(&g_abort_epoch, wc.epoch);
+              }
+              ok = false;
+              return false;
+            }
+          }
+        }
+        if (item < 0) return false;
+        if (item >= n_items) {  // cannot happen unless the ring protocol is broken
+          raise_error(LLAMA_ATTN_DEVERR_TIMEOUT);
+          atomicExch(&g_abort_epoch, wc.epoch);
+          ok = false;
+          return false;
+        }
+        I = item_of(item, p);
+        const int qi = I.q0 + r;
+        qi_c = min(qi, p.S - 1);
+        ds_i = p.doc_start ? p.doc_start[I.rowbase + qi_c] : 0;
+        qi_c += q_global(I.q0, p) - I.q0;  // from here on the row's global position
+        if (!mbar_wait(bar(B_Q_FULL), it & 1, wc)) {
+          ok = false;
+          return false;
+        }
+        // Rotate the warp's 32 Q rows two at a time: 16 lanes per row, 4 pairs
+        // per lane. A half-warp walks rows 2 apart; inside a document their
+        // positions are 2 apart too, so the (cos, sin) of the next row follow
+        // from the current ones by one rotation by 2*theta_k (angle addition,
+        // the table's row for position 2). The table is read only for the first
+        // row and where positions restart at a document start.
+        if (!p.q_rotated) {
+          const int ch = lane & 15;
+          const float4* step = p.rope_tab + 2 * 32 + 2 * ch;
+          const float4 st0 = __ldg(step), st1 = __ldg(step + 1);
+          float4 c0 = make_float4(1.f, 0.f, 1.f, 0.f), c1 = c0;
+          int pos_prev = -4;
+  #pragma unroll 4
+          for (int i = 0; i < 16; ++i) {
+            const int src = 2 * i + (lane >> 4);  // lane of the warp that owns the row
+            const int rr = wq * 32 + src;
+            const int pos = __shfl_sync(0xffffffffu, qi_c - ds_i, src);
+            if (pos == pos_prev + 2) {
+              c0 = make_float4(c0.x * st0.x - c0.y * st0.y, c0.y * st0.x + c0.x * st0.y,
+                               c0.z * st0.z - c0.w * st0.w, c0.w * st0.z + c0.z * st0.w);
+              c1 = make_float4(c1.x * st1.x - c1.y * st1.y, c1.y * st1.x + c1.x * st1.y,
+                               c1.z * st1.z - c1.w * st1.w, c1.w * st1.z + c1.z * st1.w);
+            } else {
+              const float4* tab = p.rope_tab + static_cast<int64_t>(pos) * 32 + 2 * ch;
+              c0 = __ldg(tab);
+              c1 = __ldg(tab + 1);
+            }
+            pos_prev = pos;
+            if (I.q0 + rr < p.S) {
+              uint4* ptr = reinterpret_cast<uint4*>(qtile + (ch >> 3) * HALF + sw128_off(rr, ch & 7));
+              uint4 x = *ptr;
+              x.x = rope_rotate_pair(x.x, c0.x, c0.y);
+              x.y = rope_rotate_pair(x.y, c0.z, c0.w);
+              x.z = rope_rotate_pair(x.z, c1.x, c1.y);
+              x.w = rope_rotate_pair(x.w, c1.z, c1.w);
+              *ptr = x;
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(B_Q_READY + s));
         return true;
       };
-      // The RoPE table rows an item's Q rotation will read: positions
-      // q0 - ds(q0) .. +127 and, when a document starts inside the tile, 0 .. 127.
-      auto prefetch_rows = [&](int v) {
-        if (v < 0 || v >= n_items || p.q_rotated) return;
-        const Item J = item_of(v, p);
-        const int ds0 = p.doc_start ? p.doc_start[J.rowbase + J.q0] : 0;
-        const int p0 = q_global(J.q0, p) - ds0;
-        const int n0 = min(BM, p.n_pos - p0);
-        if (n0 > 0) bulk_prefetch_l2(p.rope_tab + static_cast<int64_t>(p0) * 32, static_cast<uint32_t>(n0) * 512u);
-        if (J.ds_last > J.q0) bulk_prefetch_l2(p.rope_tab, static_cast<uint32_t>(min(BM, p.n_pos)) * 512u);
-      };
-      auto publish = [&](int k, int v) {
-        ring_item[k % kItemRing] = v;
-        __threadfence_block();
-        ring_seq[k % kItemRing] = k;
-      };
-      int it = 0, item = blockIdx.x;
-      int next_item = (item < n_items) ? atomicAdd(p.sched, 1) + static_cast<int>(gridDim.x) : n_items;
-      bool ended = false;
-      publish(0, item < n_items ? item : -1);
-      prefetch_rows(item);
-      for (;; ++it) {
-        if (it > 0 && !mbar_wait_backoff(bar(B_Q_FREE), (it - 1) & 1, wc)) {
-          ok = false;
-          break;
-        }
-        if (item >= n_items) {
-          mbar_arrive(bar(B_Q_FULL));
-          ended = true;
-          break;
-        }
-        const Item I = item_of(item, p);
-        mbar_arrive_expect_tx(bar(B_Q_FULL), static_cast<uint32_t>(p.NH) * TILE);
-        for (int s = 0; s < p.NH; ++s)
-          for (int hf = 0; hf < 2; ++hf)
-            tma_load_4d(sbase + OFF_Q + s * TILE + hf * HALF, &tm_q, bar(B_Q_FULL), hf * 64, I.h0 + s, I.q0, I.b);
-        item = next_item;
-        next_item = (item < n_items) ? atomicAdd(p.sched, 1) + static_cast<int>(gridDim.x) : n_items;
-        publish(it + 1, item < n_items ? item : -1);
-        prefetch_rows(item);
-        ok = load(false, I.g, I.kv_t0 * BN, I.b);
-        for (int j = 1; ok && j < I.n_kv; ++j)
-          ok = load(false, I.g, (I.kv_t0 + j) * BN, I.b) && load(true, I.g, (I.kv_t0 + j - 1) * BN, I.b);
-        if (ok) ok = load(true, I.g, (I.kv_t0 + I.n_kv - 1) * BN, I.b);
-        if (!ok) {
-          ++it;
-          break;
-        }
-      }
-      // Every issued load has landed before this CTA may exit (these return at
-      // once in the normal flow, where every load was consumed).
-      if (!ended && it > 0) mbar_wait(bar(B_Q_FULL), (it - 1) & 1, wc);
-      // Only the last load into a stage can still be in flight (each load
-      // waited for the stage to be emptied), so the latest phase of each
-      // kind's full barrier covers every load.
-      for (int st = 0; st < NSTAGE; ++st) {
-        if ((k_any >> st) & 1u) mbar_wait(bar(B_K_FULL + st), ((k_par >> st) & 1u) ^ 1u, wc);
-        if ((v_any >> st) & 1u) mbar_wait(bar(B_V_FULL + st), ((v_par >> st) & 1u) ^ 1u, wc);
-      }
-    }
-  } else if (warp == 1 || warp == 2) {
-    // ------------------------------------------------------------ MMA issuers
-    // Per item the load order is K0, K1, V0, K2, V1, ..., K(n-1), V(n-2), V(n-1):
-    // K_j sits at ring index base + (j == 0 ? 0 : 2j - 1) and V_j at
-    // base + (j < n-1 ? 2j + 2 : 2n - 1); base advances by 2n per item.
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = umma_idesc_bf16_f32(128, 128, 0);
-      constexpr uint32_t idesc_pv = umma_idesc_bf16_f32(128, 128, 1);
-      bool ok = true;
-      uint32_t ring = 0, tiles = 0;
-      // bit st: parity of the next phase this issuer waits for on stage st's
-      // full barrier of its tile kind (K for the S issuer, V for the PV issuer)
-      uint32_t full_par = 0;
-      for (int it = 0; ok; ++it) {
-        if (!mbar_wait(bar(B_Q_FULL), it & 1, wc)) break;
-        // The PV issuer waits on Q_FULL only to learn the item id; its arrival
-        // on Q_FREE keeps the next Q load behind this wait, so its parity wait
-        // can never fall two phases behind.
-        if (warp == 2) mbar_arrive(bar(B_Q_FREE));
-        const int item = ring_item[it % kItemRing];
-        if (item < 0 || item >= n_items) break;
-        const Item I = item_of(item, p);
-        if (warp == 1) {
-          for (int s = 0; s < p.NH; ++s) ok = ok && mbar_wait(bar(B_Q_READY + s), it & 1, wc);
-          for (int j = 0; ok && j < I.n_kv; ++j) {
-            const uint32_t idx = ring + ((j == 0) ? 0u : static_cast<uint32_t>(2 * j - 1));
-            const uint32_t st = idx % NSTAGE;
-            const uint32_t T = tiles + j;
-            if (!mbar_wait(bar(B_K_FULL + static_cast<int>(st)), (full_par >> st) & 1u, wc)) {
-              ok = false;
-              break;
-            }
-            full_par ^= 1u << st;
-            const uint64_t db = kdesc(sbase + OFF_KV + st * TILE);
-            for (int s = 0; s < p.NH; ++s) {
-              if (T > 0 && !mbar_wait(bar(B_S_FREE + s), (T - 1) & 1, wc)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              const uint64_t da = kdesc(sbase + OFF_Q + s * TILE);
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t off = ((kk >> 2) * HALF + (kk & 3) * 32) >> 4;
-                tc_mma_ss(tmem + s * 128, da + off, db + off, idesc_qk, kk > 0);
-              }
-              tc_commit(bar(B_S_READY + s));
-            }
-            tc_commit(bar(B_KV_EMPTY + st));
-          }
-          tc_commit(bar(B_Q_FREE));  // the Q tiles are free once these MMAs complete
-        } else {
-          for (int j = 0; ok && j < I.n_kv; ++j) {
-            const uint32_t idx =
-                ring + ((j < I.n_kv - 1) ? static_cast<uint32_t>(2 * j + 2) : static_cast<uint32_t>(2 * I.n_kv - 1));
-            const uint32_t st = idx % NSTAGE;
-            const uint32_t T = tiles + j;
-            if (!mbar_wait(bar(B_V_FULL + static_cast<int>(st)), (full_par >> st) & 1u, wc)) {
-              ok = false;
-              break;
-            }
-            full_par ^= 1u << st;
-            const uint64_t db = vdesc(sbase + OFF_KV + st * TILE);
-            for (int s = 0; s < p.NH; ++s) {
-              if (!mbar_wait(bar(B_P_READY + s), T & 1, wc)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              const uint64_t da = kdesc(sbase + OFF_P + s * TILE);
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t aoff = ((kk >> 2) * HALF + (kk & 3) * 32) >> 4;
-                tc_mma_ss(tmem + 256 + s * 128, da + aoff, db + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
-                          (j > 0 || kk > 0) ? 1u : 0u);
-              }
-              tc_commit(bar(B_PV_DONE + s));
-            }
-            tc_commit(bar(B_KV_EMPTY + st));
-          }
-        }
-        ring += 2u * static_cast<uint32_t>(I.n_kv);
-        tiles += static_cast<uint32_t>(I.n_kv);
-      }
-      // all issued MMAs complete before TMEM may be freed
-      const int drain = (warp == 1) ? B_DRAIN : B_DRAIN_PV;
-      tc_commit(bar(drain));
-      mbar_wait(bar(drain), 0, wc);
-    }
-  } else if (warp == 3) {
-    // ------------------------------------------------------------ output stores
-    if (lane == 0) {
-      bool ok = true;
-      for (int it = 0; ok; ++it) {
-        if (!mbar_wait_backoff(bar(B_O_STAGED + 0), it & 1, wc)) break;
-        const int item = ring_item[it % kItemRing];
-        if (item < 0 || item >= n_items) break;
-        const Item I = item_of(item, p);
-        for (int s = 0; ok && s < p.NH; ++s) {
-          if (s > 0 && !mbar_wait_backoff(bar(B_O_STAGED + s), it & 1, wc)) {
-            ok = false;
-            break;
-          }
-          tma_store_4d(&tm_o, sbase + OFF_P + s * TILE, 0, I.h0 + s, I.q0, I.b);
-          tma_store_4d(&tm_o, sbase + OFF_P + s * TILE + HALF, 64, I.h0 + s, I.q0, I.b);
-          tma_store_commit();
-          tma_store_wait_read0();  // the P buffer may be rewritten from here on
-          mbar_arrive(bar(B_O_READ + s));
-        }
-      }
-      tma_store_wait0();
-    }
-  } else if (warp >= 4 && (warp - 4) / 4 < p.NH) {
-    // ------------------------------------------------------------ softmax
-    const int s = (warp - 4) >> 2;
-    const int wq = warp & 3;
-    const int r = wq * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + lane_off + s * 128;
-    const uint32_t tO = tmem + lane_off + 256 + s * 128;
-    uint8_t* qtile = smem + OFF_Q + s * TILE;
-    uint8_t* ptile = smem + OFF_P + s * TILE;
-    const float sl2 = p.scale_log2;
-    bool ok = true;
-    uint32_t tiles = 0;
-    Item I;
-    int qi_c = 0, ds_i = 0;  // global position of this thread's (clamped) row; its document start
-    // Starts item `it`: reads its id from the ring, loads its row data, waits for
-    // its Q tile and rotates this thread's row in place. False at the end of the
-    // items (or on a timeout, which also clears ok).
-    auto begin_item = [&](int it) -> bool {
-      int item = -1;
-      {
-        const unsigned long long t0 = global_ns();
-        for (uint32_t k = 0;; ++k) {
-          if (ring_seq[it % kItemRing] == it) {
-            __threadfence_block();  // the item id was written before its sequence number
-            item = ring_item[it % kItemRing];
-            break;
-          }
-          if ((k & 63u) == 63u && (wc.aborted() || global_ns() - t0 > kWaitTimeoutNs)) {
-            if (!wc.aborted()) {
-              raise_error(LLAMA_ATTN_DEVERR_TIMEOUT);
-              atomicExch(&g_abort_epoch, wc.epoch);
-            }
-            ok = false;
-            return false;
-          }
-        }
-      }
-      if (item < 0) return false;
-      if (item >= n_items) {  // cannot happen unless the ring protocol is broken
-        raise_error(LLAMA_ATTN_DEVERR_TIMEOUT);
-        atomicExch(&g_abort_epoch, wc.epoch);
-        ok = false;
-        return false;
-      }
-      I = item_of(item, p);
-      const int qi = I.q0 + r;
-      qi_c = min(qi, p.S - 1);
-      ds_i = p.doc_start ? p.doc_start[I.rowbase + qi_c] : 0;
-      qi_c += q_global(I.q0, p) - I.q0;  // from here on the row's global position
-      if (!mbar_wait(bar(B_Q_FULL), it & 1, wc)) {
-        ok = false;
-        return false;
-      }
-      // Rotate the warp's 32 Q rows two at a time: 16 lanes per row, 4 pairs
-      // per lane. A half-warp walks rows 2 apart; inside a document their
-      // positions are 2 apart too, so the (cos, sin) of the next row follow
-      // from the current ones by one rotation by 2*theta_k (angle addition,
-      // the table's row for position 2). The table is read only for the first
-      // row and where positions restart at a document start.
-      if (!p.q_rotated) {
-        const int ch = lane & 15;
-        const float4* step = p.rope_tab + 2 * 32 + 2 * ch;
-        const float4 st0 = __ldg(step), st1 = __ldg(step + 1);
-        float4 c0 = make_float4(1.f, 0.f, 1.f, 0.f), c1 = c0;
-        int pos_prev = -4;
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-          const int src = 2 * i + (lane >> 4);  // lane of the warp that owns the row
-          const int rr = wq * 32 + src;
-          const int pos = __shfl_sync(0xffffffffu, qi_c - ds_i, src);
-          if (pos == pos_prev + 2) {
-            c0 = make_float4(c0.x * st0.x - c0.y * st0.y, c0.y * st0.x + c0.x * st0.y,
-                             c0.z * st0.z - c0.w * st0.w, c0.w * st0.z + c0.z * st0.w);
-            c1 = make_float4(c1.x * st1.x - c1.y * st1.y, c1.y * st1.x + c1.x * st1.y,
-                             c1.z * st1.z - c1.w * st1.w, c1.w * st1.z + c1.z * st1.w);
-          } else {
-            const float4* tab = p.rope_tab + static_cast<int64_t>(pos) * 32 + 2 * ch;
-            c0 = __ldg(tab);
-            c1 = __ldg(tab + 1);
-          }
-          pos_prev = pos;
-          if (I.q0 + rr < p.S) {
-            uint4* ptr = reinterpret_cast<uint4*>(qtile + (ch >> 3) * HALF + sw128_off(rr, ch & 7));
-            uint4 x = *ptr;
-            x.x = rope_rotate_pair(x.x, c0.x, c0.y);
-            x.y = rope_rotate_pair(x.y, c0.z, c0.w);
-            x.z = rope_rotate_pair(x.z, c1.x, c1.y);
-            x.w = rope_rotate_pair(x.w, c1.z, c1.w);
-            *ptr = x;
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bar(B_Q_READY + s));
-      return true;
-    };
 
-    bool more = begin_item(0);
-    const bool begin_ok_first = more;
-    for (int it = 0; ok && more; ++it) {
-      float m = -INFINITY;  // reference max, in log2 units of the scaled score
-      float l = 0.f;
-      for (int j = 0; j < I.n_kv; ++j) {
-        const int kb = (I.kv_t0 + j) * BN;
-        const uint32_t T = tiles + j;
-        if (!mbar_wait(bar(B_S_READY + s), T & 1, wc)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        uint32_t sr[128];
-        tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-        tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
-        tc_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(B_S_FREE + s));
-
-        float sv[128];
-#pragma unroll
-        for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c]);
-        if (j == I.n_kv - 1 || kb < I.ds_last) {  // the diagonal tile, or a document starts in it
-          const int lo = ds_i - kb, hi = qi_c - kb;
-#pragma unroll
-          for (int c = 0; c < 128; ++c) sv[c] = (c < lo || c > hi) ? -INFINITY : sv[c];
-        }
-        // four running maxima over columns a, a+4, ..., a+124 (a = 0..3)
-        float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
-#pragma unroll
-        for (int c = 4; c <= 116; c += 8) {
-          mx0 = max3(mx0, sv[c], sv[c + 4]);
-          mx1 = max3(mx1, sv[c + 1], sv[c + 5]);
-          mx2 = max3(mx2, sv[c + 2], sv[c + 6]);
-          mx3 = max3(mx3, sv[c + 3], sv[c + 7]);
-        }
-        mx0 = fmaxf(mx0, sv[124]);
-        mx1 = fmaxf(mx1, sv[125]);
-        mx2 = fmaxf(mx2, sv[126]);
-        mx3 = fmaxf(mx3, sv[127]);
-        const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-        const float m_new = fmaxf(m, mt);
-        const bool resc = m_new > m + kRescaleLog2;
-        float alpha = 1.f;
-        if (resc) {
-          alpha = ex2_approx(m - m_new);
-          m = m_new;
-        }
-        const float neg_m = (m == -INFINITY) ? 0.f : -m;
-        uint32_t pk[64];
-        // x = s * log2(e)/sqrt(D) - m and the running row sum in packed fp32 pairs
-        const uint64_t sl2x2 = f2_pack(sl2, sl2), negmx2 = f2_pack(neg_m, neg_m);
-        uint64_t rsa = f2_pack(0.f, 0.f), rsb = rsa;
-#pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sl2x2, negmx2), x0, x1);
-          // one pair in eight goes through the FMA-pipe polynomial, the rest through
-          // MUFU (a larger share measured slower: it raises register pressure)
-          const bool poly = (c & 14) == 14;
-          const float p0 = poly ? ex2_poly(x0) : ex2_approx(x0);
-          const float p1 = poly ? ex2_poly(x1) : ex2_approx(x1);
-          if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));
-          else rsa = f2_add(rsa, f2_pack(p0, p1));
-          pk[c >> 1] = pack_bf16x2(p0, p1);
-        }
-        float rs0, rs1, rs2, rs3;
-        f2_unpack(rsa, rs0, rs1);
-        f2_unpack(rsb, rs2, rs3);
-        l = l * alpha + ((rs0 + rs2) + (rs1 + rs3));
-
-        if (j > 0) {
-          if (!mbar_wait(bar(B_PV_DONE + s), (T - 1) & 1, wc)) {
+      bool more = begin_item(0);
+      const bool begin_ok_first = more;
+      for (int it = 0; ok && more; ++it) {
+        float m = -INFINITY;  // reference max, in log2 units of the scaled score
+        float l = 0.f;
+        for (int j = 0; j < I.n_kv; ++j) {
+          const int kb = (I.kv_t0 + j) * BN;
+          const uint32_t T = tiles + j;
+          if (!mbar_wait(bar(B_S_READY + s), T & 1, wc)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          if (__any_sync(0xffffffffu, resc)) {
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-              uint32_t o[32];
-              tmem_ld32(tO + ch * 32, o);
-              tc_wait_ld();
-#pragma unroll
-              for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
-              tmem_st32(tO + ch * 32, o);
-            }
-            tc_wait_st();
+          uint32_t sr[128];
+          tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+          tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+          tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+          tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+          tc_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar(B_S_FREE + s));
+
+          float sv[128];
+  #pragma unroll
+          for (int c = 0; c < 128; ++c) sv[c] = __uint_as_float(sr[c]);
+          if (j == I.n_kv - 1 || kb < I.ds_last) {  // the diagonal tile, or a document starts in it
+            const int lo = ds_i - kb, hi = qi_c - kb;
+  #pragma unroll
+            for (int c = 0; c < 128; ++c) sv[c] = (c < lo || c > hi) ? -INFINITY : sv[c];
           }
-        } else if (it > 0 && !mbar_wait(bar(B_O_READ + s), (it - 1) & 1, wc)) {
-          // the previous item's output left the P buffer
+          // four running maxima over columns a, a+4, ..., a+124 (a = 0..3)
+          float mx0 = sv[0], mx1 = sv[1], mx2 = sv[2], mx3 = sv[3];
+  #pragma unroll
+          for (int c = 4; c <= 116; c += 8) {
+            mx0 = max3(mx0, sv[c], sv[c + 4]);
+            mx1 = max3(mx1, sv[c + 1], sv[c + 5]);
+            mx2 = max3(mx2, sv[c + 2], sv[c + 6]);
+            mx3 = max3(mx3, sv[c + 3], sv[c + 7]);
+          }
+          mx0 = fmaxf(mx0, sv[124]);
+          mx1 = fmaxf(mx1, sv[125]);
+          mx2 = fmaxf(mx2, sv[126]);
+          mx3 = fmaxf(mx3, sv[127]);
+          const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+          const float m_new = fmaxf(m, mt);
+          const bool resc = m_new > m + kRescaleLog2;
+          float alpha = 1.f;
+          if (resc) {
+            alpha = ex2_approx(m - m_new);
+            m = m_new;
+          }
+          const float neg_m = (m == -INFINITY) ? 0.f : -m;
+          uint32_t pk[64];
+          // x = s * log2(e)/sqrt(D) - m and the running row sum in packed fp32 pairs
+          const uint64_t sl2x2 = f2_pack(sl2, sl2), negmx2 = f2_pack(neg_m, neg_m);
+          uint64_t rsa = f2_pack(0.f, 0.f), rsb = rsa;
+  #pragma unroll
+          for (int c = 0; c < 128; c += 2) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sl2x2, negmx2), x0, x1);
+            // one pair in four goes through the FMA-pipe polynomial, the rest through
+            // MUFU (a larger share measured slower: the polynomial's FMA and ALU
+            // instructions cost more issue time than the MUFU time they save)
+            const bool poly = (c & 6) == 6;
+            const float p0 = poly ? ex2_poly(x0) : ex2_approx(x0);
+            const float p1 = poly ? ex2_poly(x1) : ex2_approx(x1);
+            if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));
+            else rsa = f2_add(rsa, f2_pack(p0, p1));
+            pk[c >> 1] = pack_bf16x2(p0, p1);
+          }
+          float rs0, rs1, rs2, rs3;
+          f2_unpack(rsa, rs0, rs1);
+          f2_unpack(rsb, rs2, rs3);
+          l = l * alpha + ((rs0 + rs2) + (rs1 + rs3));
+
+          if (j > 0) {
+            if (!mbar_wait(bar(B_PV_DONE + s), (T - 1) & 1, wc)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, resc)) {
+  #pragma unroll
+              for (int ch = 0; ch < 4; ++ch) {
+                uint32_t o[32];
+                tmem_ld32(tO + ch * 32, o);
+                tc_wait_ld();
+  #pragma unroll
+                for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * alpha);
+                tmem_st32(tO + ch * 32, o);
+              }
+              tc_wait_st();
+            }
+          } else if (it > 0 && !mbar_wait(bar(B_O_READ + s), (it - 1) & 1, wc)) {
+            // the previous item's output left the P buffer
+            ok = false;
+            break;
+          }
+  #pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            uint4 w;
+            w.x = pk[4 * c];
+            w.y = pk[4 * c + 1];
+            w.z = pk[4 * c + 2];
+            w.w = pk[4 * c + 3];
+            *reinterpret_cast<uint4*>(ptile + (c >> 3) * HALF + sw128_off(r, c & 7)) = w;
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(bar(B_P_READY + s));
+        }
+        if (!ok) break;
+
+        // The next item's Q rotation overlaps the last PV of this one.
+        const Item cur = I;
+        const float l_cur = l;
+        more = begin_item(it + 1);
+        if (!ok) break;
+
+        // ---- epilogue: O / l -> bf16 -> P buffer; warp 3 stores it with TMA
+        const uint32_t T_last = tiles + cur.n_kv - 1;
+        if (!mbar_wait(bar(B_PV_DONE + s), T_last & 1, wc)) {
           ok = false;
           break;
         }
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          uint4 w;
-          w.x = pk[4 * c];
-          w.y = pk[4 * c + 1];
-          w.z = pk[4 * c + 2];
-          w.w = pk[4 * c + 3];
-          *reinterpret_cast<uint4*>(ptile + (c >> 3) * HALF + sw128_off(r, c & 7)) = w;
+        tc_fence_after();
+        const float inv_l = 1.f / l_cur;
+  #pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          uint32_t o[32];
+          tmem_ld32(tO + ch * 32, o);
+          tc_wait_ld();
+  #pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[8 * c4 + 0]) * inv_l, __uint_as_float(o[8 * c4 + 1]) * inv_l);
+            w.y = pack_bf16x2(__uint_as_float(o[8 * c4 + 2]) * inv_l, __uint_as_float(o[8 * c4 + 3]) * inv_l);
+            w.z = pack_bf16x2(__uint_as_float(o[8 * c4 + 4]) * inv_l, __uint_as_float(o[8 * c4 + 5]) * inv_l);
+            w.w = pack_bf16x2(__uint_as_float(o[8 * c4 + 6]) * inv_l, __uint_as_float(o[8 * c4 + 7]) * inv_l);
+            const int d = ch * 32 + c4 * 8;
+            *reinterpret_cast<uint4*>(ptile + (d >> 6) * HALF + sw128_off(r, (d & 63) >> 3)) = w;
+          }
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(bar(B_P_READY + s));
-      }
-      if (!ok) break;
-
-      // The next item's Q rotation overlaps the last PV of this one.
-      const Item cur = I;
-      const float l_cur = l;
-      more = begin_item(it + 1);
-      if (!ok) break;
-
-      // ---- epilogue: O / l -> bf16 -> P buffer; warp 3 stores it with TMA
-      const uint32_t T_last = tiles + cur.n_kv - 1;
-      if (!mbar_wait(bar(B_PV_DONE + s), T_last & 1, wc)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      const float inv_l = 1.f / l_cur;
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t o[32];
-        tmem_ld32(tO + ch * 32, o);
-        tc_wait_ld();
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(o[8 * c4 + 0]) * inv_l, __uint_as_float(o[8 * c4 + 1]) * inv_l);
-          w.y = pack_bf16x2(__uint_as_float(o[8 * c4 + 2]) * inv_l, __uint_as_float(o[8 * c4 + 3]) * inv_l);
-          w.z = pack_bf16x2(__uint_as_float(o[8 * c4 + 4]) * inv_l, __uint_as_float(o[8 * c4 + 5]) * inv_l);
-          w.w = pack_bf16x2(__uint_as_float(o[8 * c4 + 6]) * inv_l, __uint_as_float(o[8 * c4 + 7]) * inv_l);
-          const int d = ch * 32 + c4 * 8;
-          *reinterpret_cast<uint4*>(ptile + (d >> 6) * HALF + sw128_off(r, (d & 63) >> 3)) = w;
+        mbar_arrive(bar(B_O_STAGED + s));
+        if (p.lse != nullptr && cur.q0 + r < p.S)  // natural log: ln 2 * (m + log2 l)
+          p.lse[(cur.rowbase + cur.q0 + r) * p.Hq + cur.h0 + s] = 0.69314718055994531f * (m + log2f(l_cur));
+        tiles += static_cast<uint32_t>(cur.n_kv);
+        if (!more && ok && s == 0) {
+          // tell the store warp the items are done, once it has read the last output
+          mbar_wait(bar(B_O_READ + 0), it & 1, wc);
+          mbar_arrive(bar(B_O_STAGED + 0));
         }
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar(B_O_STAGED + s));
-      if (p.lse != nullptr && cur.q0 + r < p.S)  // natural log: ln 2 * (m + log2 l)
-        p.lse[(cur.rowbase + cur.q0 + r) * p.Hq + cur.h0 + s] = 0.69314718055994531f * (m + log2f(l_cur));
-      tiles += static_cast<uint32_t>(cur.n_kv);
-      if (!more && ok && s == 0) {
-        // tell the store warp the items are done, once it has read the last output
-        mbar_wait(bar(B_O_READ + 0), it & 1, wc);
-        mbar_arrive(bar(B_O_STAGED + 0));
-      }
+      if (ok && s == 0 && !begin_ok_first) mbar_arrive(bar(B_O_STAGED + 0));  // no items at all
     }
-    if (ok && s == 0 && !begin_ok_first) mbar_arrive(bar(B_O_STAGED + 0));  // no items at all
   }
 
   tc_fence_before();

@@ -12,12 +12,14 @@ every wait is satisfied with exactly k+1 phases completed and that every role
 finishes.
 
 What it shows:
-  * the kernel's protocol (one full barrier per ring stage and tile kind,
-    each waited by its one consumer in consecutive phases) is correct with
+  * the kernel's protocol (K tiles in a ring of two stages, V tiles in a
+    ring of one, each stage with its own full and empty barriers, each full
+    barrier waited in consecutive phases by its one consumer) is correct with
     asynchronous completions landing in any order: it does not rely on TMA
     loads completing in the order they were issued, which PTX does not
-    promise;
-  * the earlier form, where K and V tiles shared one full barrier per stage
+    promise; so is the previous form (one shared ring, full barriers split by
+    tile kind);
+  * the earliest form, where K and V tiles shared one full barrier per stage
     and each MMA issuer waited only on its own tiles' phases, relied on that
     order: a later load landing first lets a wait pass early;
   * the S issuer's wait for the softmax's Q-ready arrival is needed even
@@ -65,10 +67,14 @@ def v_index(j, n):
     return 2 * j + 2 if j < n - 1 else 2 * n - 1
 
 
-def roles(items, q_free_count, s_waits_q_ready, split_full=False):
+def roles(items, q_free_count, s_waits_q_ready, split_full=False, rings=None):
     """Generators yielding ('wait', name, phase) / ('arrive', name) /
-    ('async', name) steps, one per role; the item list ends with a sentinel."""
+    ('async', name) steps, one per role; the item list ends with a sentinel.
+    rings=(NK, NV): K and V tiles in rings of their own (NK and NV stages),
+    each with its own full and empty barriers."""
     NH = 2
+    if rings is not None:
+        return _ring_roles(items, q_free_count, s_waits_q_ready, rings)
 
     def producer():
         idx = 0
@@ -183,9 +189,80 @@ def roles(items, q_free_count, s_waits_q_ready, split_full=False):
             "softmax0": softmax(0), "softmax1": softmax(1)}
 
 
+def _ring_roles(items, q_free_count, s_waits_q_ready, rings):
+    NH = 2
+    NK, NV = rings
+    base = roles(items, q_free_count, s_waits_q_ready)  # store and softmax roles are unchanged
+
+    def producer():
+        kt = vt = 0
+        for it, n in enumerate(items + [None]):
+            if it > 0:
+                yield ("wait", "Q_FREE", it - 1)
+            if n is None:
+                yield ("arrive", "Q_FULL")
+                return
+            yield ("async", "Q_FULL")
+            for kind, _ in kv_ring(n):
+                if kind == "K":
+                    st, use = kt % NK, kt // NK
+                    if use > 0:
+                        yield ("wait", f"K_EMPTY{st}", use - 1)
+                    yield ("async", f"K_FULL{st}")
+                    kt += 1
+                else:
+                    st, use = vt % NV, vt // NV
+                    if use > 0:
+                        yield ("wait", f"V_EMPTY{st}", use - 1)
+                    yield ("async", f"V_FULL{st}")
+                    vt += 1
+
+    def s_issuer():
+        tiles = 0
+        for it, n in enumerate(items + [None]):
+            yield ("wait", "Q_FULL", it)
+            if n is None:
+                return
+            if s_waits_q_ready:
+                for s in range(NH):
+                    yield ("wait", f"Q_READY{s}", it)
+            for j in range(n):
+                T = tiles + j
+                yield ("wait", f"K_FULL{T % NK}", T // NK)
+                for s in range(NH):
+                    if T > 0:
+                        yield ("wait", f"S_FREE{s}", T - 1)
+                    yield ("async", f"S_READY{s}")
+                yield ("async", f"K_EMPTY{T % NK}")
+            yield ("async", "Q_FREE")
+            tiles += n
+
+    def pv_issuer():
+        tiles = 0
+        for it, n in enumerate(items + [None]):
+            yield ("wait", "Q_FULL", it)
+            if q_free_count == 2:
+                yield ("arrive", "Q_FREE")
+            if n is None:
+                return
+            for j in range(n):
+                T = tiles + j
+                yield ("wait", f"V_FULL{T % NV}", T // NV)
+                for s in range(NH):
+                    yield ("wait", f"P_READY{s}", T)
+                    yield ("async", f"PV_DONE{s}")
+                yield ("async", f"V_EMPTY{T % NV}")
+            tiles += n
+
+    base.update(producer=producer(), s_issuer=s_issuer(), pv_issuer=pv_issuer())
+    return base
+
+
 def barriers(q_free_count):
     b = {"Q_FULL": Barrier(1), "Q_FREE": Barrier(q_free_count)}
     for st in range(NSTAGE):
+        for name in ("K_FULL", "K_EMPTY", "V_FULL", "V_EMPTY"):
+            b[f"{name}{st}"] = Barrier(1)
         b[f"KV_FULL{st}"] = Barrier(1)
         b[f"FULL_K{st}"] = Barrier(1)
         b[f"FULL_V{st}"] = Barrier(1)
@@ -199,13 +276,13 @@ def barriers(q_free_count):
 
 
 def simulate(items, seed, q_free_count=2, s_waits_q_ready=True, in_order=True, split_full=False,
-             max_steps=200000):
+             max_steps=200000, rings=None):
     """in_order: each asynchronous source completes in the order it issued
     (the producer's TMA loads; each MMA issuer's commits); sources interleave
     freely. in_order=False lets any in-flight completion land first."""
     rng = random.Random(seed)
     bars = barriers(q_free_count)
-    gens = roles(items, q_free_count, s_waits_q_ready, split_full)
+    gens = roles(items, q_free_count, s_waits_q_ready, split_full, rings)
     current = {name: next(g, None) for name, g in gens.items()}
     inflight = []  # (source, barrier) of completions not yet landed (MMA commits, TMA bytes)
     for _ in range(max_steps):
@@ -255,9 +332,18 @@ def _random_items(seed):
 
 @pytest.mark.parametrize("seed", range(80))
 def test_committed_protocol_needs_no_completion_order(seed):
-    """The kernel's protocol: split full barriers, Q-ready handshake kept."""
-    simulate(_random_items(seed), seed, in_order=False, split_full=True)
-    simulate(_random_items(seed), seed + 7, in_order=True, split_full=True)
+    """The kernel's protocol: separate K (two stages) and V (one stage) rings,
+    Q-ready handshake kept."""
+    simulate(_random_items(seed), seed, in_order=False, rings=(2, 1))
+    simulate(_random_items(seed), seed + 7, in_order=True, rings=(2, 1))
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_other_ring_splits_and_the_split_barrier_form(seed):
+    """The other division of the three stages, and the previous revision's
+    shared ring with full barriers split by tile kind, are correct too."""
+    simulate(_random_items(seed), seed + 11, in_order=False, rings=(1, 2))
+    simulate(_random_items(seed), seed + 13, in_order=False, split_full=True)
 
 
 def test_shared_full_barriers_rely_on_tma_completion_order():

@@ -1,4 +1,4 @@
-"""The FMA-pipe 2^x used for one softmax exponential in eight: its
+"""The FMA-pipe 2^x used for one softmax exponential pair in four: its
 constants come from the committed fit, and the float32 evaluation (range
 reduction + cubic + exponent add) stays within 1e-4 relative error of exp2."""
 import os
