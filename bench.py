@@ -729,6 +729,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     prefill_names = [n for n, x in W.WORKLOADS.items() if isinstance(x, W.PrefillWorkload) and x.dtype == "bf16"]
+    prefill_names += list(W.CAPTURE_WORKLOADS)  # smaller launches for counter captures only
     ap.add_argument("--workload", default=W.LONG_128K.name, choices=prefill_names,
                     help="the headline prefill workload (the line's value)")
     ap.add_argument("--extra-workloads", default=",".join([W.PACKED_8B.name, W.PACKED_405B.name]),
@@ -751,7 +752,7 @@ def main():
     ap.add_argument("--cp", action="store_true",
                     help="context-parallel prefill of the workload over the GPUs (strong scaling)")
     args = ap.parse_args()
-    w = W.WORKLOADS[args.workload]
+    w = W.WORKLOADS.get(args.workload) or W.CAPTURE_WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, w)
     else:

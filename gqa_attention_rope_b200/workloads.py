@@ -72,6 +72,12 @@ DECODE_70B = DecodeWorkload("llama70b_decode_B64_Hq64_Hkv8_D128_len1024-32768", 
 
 WORKLOADS = {w.name: w for w in (TINY_F32, PACKED_8B, PACKED_405B, LONG_128K, DECODE_70B)}
 
+# A shorter single-document prefill with the 128K workload's head layout, used
+# only where hardware-counter captures need a smaller launch of the same
+# kernel; it is not one of the measured workloads.
+LONG_32K_CAPTURE = PrefillWorkload("long32k_B1_S32768_Hq32_Hkv8_D128_causal", 4, 1, 32768, 32, 8, 128, "bf16", None)
+CAPTURE_WORKLOADS = {LONG_32K_CAPTURE.name: LONG_32K_CAPTURE}
+
 
 def draw_doc_lengths(gen: torch.Generator, S: int, lo: int, hi: int) -> list:
     """Uniform integer document lengths in [lo, hi] filling one row of S tokens."""
