@@ -447,6 +447,9 @@ int prefill_bf16_launch(const llama_attn_bf16* q, const llama_attn_bf16* k, cons
   p.q_pos_a = qc.q_pos_a;
   p.q_pos_b = qc.q_pos_b;
   p.q_rotated = prerotated ? 1 : 0;
+  // Keys and values (rotated K and V) well beyond the 126 MB L2: run the items
+  // KV group by KV group so the groups' tiles are read from DRAM about once.
+  p.kv_major = (static_cast<int64_t>(B) * Skv * Hkv * 128 * 2 * 2 > (int64_t(256) << 20)) ? 1 : 0;
   p.doc_start = doc_start;
   p.rope_tab = tab4;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));

@@ -57,7 +57,7 @@ constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_KV = OFF_Q + 2 * TILE;
 constexpr uint32_t OFF_P = OFF_KV + NSTAGE * TILE;
 constexpr uint32_t OFF_BAR = OFF_P + 2 * TILE;
-constexpr uint32_t SMEM_USED = OFF_BAR + 512;
+constexpr uint32_t SMEM_USED = OFF_BAR + 1024;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;
 constexpr int NTHREADS = 384;
 constexpr uint32_t TMEM_COLS = 512;
@@ -92,6 +92,12 @@ enum : int {
 };
 constexpr int kItemRing = 8;
 static_assert(N_BARS * 8 + 8 + 8 * kItemRing <= 512, "barrier area, TMEM address and item ring");
+// Each ring slot also holds its item's fields, computed once by the producer.
+struct ItemSlot {
+  int b, h0, g, q0, ds_last, kv_t0, n_kv, pad;
+};
+constexpr uint32_t OFF_SLOTS = 512;  // from OFF_BAR
+static_assert(OFF_SLOTS + sizeof(ItemSlot) * kItemRing <= 1024, "item slots");
 
 struct Params {
   int B, S, Hq, Hkv, G, NH, n_qt, n_hp;
@@ -102,6 +108,7 @@ struct Params {
   // of 128; S when all rows form one chunk). Both 0 for a plain prefill.
   int q_split, q_pos_a, q_pos_b;
   int q_rotated;             // 1: q arrives already rotated (no in-kernel rotation, no table)
+  int kv_major;              // 1: items run KV group by KV group (keys and values far larger than L2)
   const int32_t* doc_start;  // [B*S] row-local document start, or null (one document per row)
   const float4* rope_tab;    // (cos, sin) pairs, 64 per position, as float4 = 2 pairs
   int* sched;                // work-item counter, zero at launch
@@ -128,12 +135,28 @@ __device__ __forceinline__ int q_global(int q0, const Params& p) {
 
 __device__ __forceinline__ Item item_of(int item, const Params& p) {
   Item it;
-  const int per_rank = p.B * p.n_hp;
-  const int qt = p.n_qt - 1 - item / per_rank;
-  const int rem = item % per_rank;
-  it.b = rem / p.n_hp;
-  it.h0 = (rem % p.n_hp) * p.NH;
-  it.g = it.h0 / p.G;
+  int qt;
+  if (p.kv_major) {
+    // By (batch row, KV group) block, inside a block from the last (heaviest)
+    // query tile down, head pair by head pair: the CTAs at work at any time
+    // read one KV group's keys and values, which then stay in L2.
+    const int pg = p.G / p.NH;  // head pairs (or single heads) per KV group
+    const int per_blk = p.n_qt * pg;
+    const int blk = item / per_blk, rem = item % per_blk;
+    it.b = blk / p.Hkv;
+    it.g = blk % p.Hkv;
+    qt = p.n_qt - 1 - rem / pg;
+    it.h0 = (it.g * pg + rem % pg) * p.NH;
+  } else {
+    // Heaviest first: the last query tile of every batch row and head pair,
+    // then the one before, ... (longest-processing-time-first)
+    const int per_rank = p.B * p.n_hp;
+    qt = p.n_qt - 1 - item / per_rank;
+    const int rem = item % per_rank;
+    it.b = rem / p.n_hp;
+    it.h0 = (rem % p.n_hp) * p.NH;
+    it.g = it.h0 / p.G;
+  }
   it.q0 = qt * BM;
   const int q_last = min(it.q0 + BM - 1, p.S - 1);
   it.rowbase = static_cast<int64_t>(it.b) * p.S;
@@ -167,6 +190,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // item, then the sequence number; readers poll the sequence number.
   volatile int* ring_item = reinterpret_cast<volatile int*>(smem + OFF_BAR + 8 * N_BARS + 8);
   volatile int* ring_seq = ring_item + kItemRing;
+  volatile ItemSlot* slots = reinterpret_cast<volatile ItemSlot*>(smem + OFF_BAR + OFF_SLOTS);
+  // The item published in ring slot k (read once its sequence number, or a
+  // barrier phase that follows the publication, has been seen).
+  auto slot_item = [&](int k) -> Item {
+    const volatile ItemSlot& q = slots[k % kItemRing];
+    Item it;
+    it.b = q.b;
+    it.h0 = q.h0;
+    it.g = q.g;
+    it.q0 = q.q0;
+    it.ds_last = q.ds_last;
+    it.kv_t0 = q.kv_t0;
+    it.n_kv = q.n_kv;
+    it.rowbase = static_cast<int64_t>(it.b) * p.S;
+    return it;
+  };
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * static_cast<uint32_t>(i); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -256,6 +295,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (J.ds_last > J.q0) bulk_prefetch_l2(p.rope_tab, static_cast<uint32_t>(min(BM, p.n_pos)) * 512u);
         };
         auto publish = [&](int k, int v) {
+          if (v >= 0 && v < n_items) {
+            const Item J = item_of(v, p);
+            volatile ItemSlot& q = slots[k % kItemRing];
+            q.b = J.b;
+            q.h0 = J.h0;
+            q.g = J.g;
+            q.q0 = J.q0;
+            q.ds_last = J.ds_last;
+            q.kv_t0 = J.kv_t0;
+            q.n_kv = J.n_kv;
+          }
           ring_item[k % kItemRing] = v;
           __threadfence_block();
           ring_seq[k % kItemRing] = k;
@@ -275,7 +325,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             ended = true;
             break;
           }
-          const Item I = item_of(item, p);
+          const Item I = slot_item(it);
           mbar_arrive_expect_tx(bar(B_Q_FULL), static_cast<uint32_t>(p.NH) * TILE);
           for (int s = 0; s < p.NH; ++s)
             for (int hf = 0; hf < 2; ++hf)
@@ -321,7 +371,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (warp == 2) mbar_arrive(bar(B_Q_FREE));
           const int item = ring_item[it % kItemRing];
           if (item < 0 || item >= n_items) break;
-          const Item I = item_of(item, p);
+          const Item I = slot_item(it);
           if (warp == 1) {
             for (int s = 0; s < p.NH; ++s) ok = ok && mbar_wait(bar(B_Q_READY + s), it & 1, wc);
             for (int j = 0; ok && j < I.n_kv; ++j) {
@@ -391,7 +441,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!mbar_wait_backoff(bar(B_O_STAGED + 0), it & 1, wc)) break;
           const int item = ring_item[it % kItemRing];
           if (item < 0 || item >= n_items) break;
-          const Item I = item_of(item, p);
+          const Item I = slot_item(it);
           for (int s = 0; ok && s < p.NH; ++s) {
             if (s > 0 && !mbar_wait_backoff(bar(B_O_STAGED + s), it & 1, wc)) {
               ok = false;
@@ -454,7 +504,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ok = false;
           return false;
         }
-        I = item_of(item, p);
+        I = slot_item(it);
         const int qi = I.q0 + r;
         qi_c = min(qi, p.S - 1);
         ds_i = p.doc_start ? p.doc_start[I.rowbase + qi_c] : 0;
@@ -567,10 +617,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int c = 0; c < 128; c += 2) {
             float x0, x1;
             f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sl2x2, negmx2), x0, x1);
-            // one pair in four goes through the FMA-pipe polynomial, the rest through
-            // MUFU (a larger share measured slower: the polynomial's FMA and ALU
-            // instructions cost more issue time than the MUFU time they save)
-            const bool poly = (c & 6) == 6;
+            // one pair in eight goes through the FMA-pipe polynomial, the rest
+            // through MUFU (with the register split, 1/8 and 1/4 measured best;
+            // larger shares cost more FMA and ALU issue than the MUFU time saved)
+            const bool poly = (c & 14) == 14;
             const float p0 = poly ? ex2_poly(x0) : ex2_approx(x0);
             const float p1 = poly ? ex2_poly(x1) : ex2_approx(x1);
             if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));
