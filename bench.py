@@ -306,37 +306,63 @@ def measure_prefill(args, la, dev, w, world, rank, peaks, cpu_seconds, steps):
     sustained = kernel_ms * steps / 1e3 > SUSTAINED_AFTER_S
     peak = tc_sust if sustained else tc_peak
 
-    # end to end through the public API: pinned host inputs -> device -> call -> host result
+    # End to end through the public API, as a serving loop runs it: every step
+    # uploads its own q, k, v (and offsets) from pinned host memory and
+    # downloads its output, on two copy streams, with double-buffered device
+    # tensors, so the upload of step i+1 and the download of step i-1 overlap
+    # the kernels of step i. The timed region runs from the first upload to
+    # the last download.
     hq, hk, hv = (inp[n].pin_memory() for n in ("q", "k", "v"))
     hoffs = inp["doc_offsets"].pin_memory() if inp["doc_offsets"] is not None else None
-    hout = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-    dq, dk, dv, dout = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v), torch.empty_like(q)
-    doffs = torch.empty_like(offs) if offs is not None else None
+    houts = [torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(2)]
+    bufs = [dict(q=torch.empty_like(q), k=torch.empty_like(k), v=torch.empty_like(v), o=torch.empty_like(q),
+                 offs=torch.empty_like(offs) if offs is not None else None) for _ in range(2)]
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
 
-    def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        if doffs is not None:
-            doffs.copy_(hoffs, non_blocking=True)
-        la.llama_attn_prefill(dq, dk, dv, out=dout, doc_offsets=doffs, rope_theta=w.rope_theta)
-        hout.copy_(dout, non_blocking=True)
+    def e2e_run(n):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        up_ev = [torch.cuda.Event() for _ in range(n)]
+        comp_ev = [torch.cuda.Event() for _ in range(n)]
+        down_ev = [torch.cuda.Event() for _ in range(n)]
+        t0.record(stream)
+        up.wait_event(t0)
+        for i in range(n):
+            b = bufs[i % 2]
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(comp_ev[i - 2])  # the kernels of step i-2 have read this buffer
+                b["q"].copy_(hq, non_blocking=True)
+                b["k"].copy_(hk, non_blocking=True)
+                b["v"].copy_(hv, non_blocking=True)
+                if b["offs"] is not None:
+                    b["offs"].copy_(hoffs, non_blocking=True)
+                up_ev[i].record(up)
+            stream.wait_event(up_ev[i])
+            if i >= 2:
+                stream.wait_event(down_ev[i - 2])  # step i-2's output has left this buffer
+            la.llama_attn_prefill(b["q"], b["k"], b["v"], out=b["o"], doc_offsets=b["offs"],
+                                  rope_theta=w.rope_theta, stream=stream)
+            comp_ev[i].record(stream)
+            with torch.cuda.stream(down):
+                down.wait_event(comp_ev[i])
+                houts[i % 2].copy_(b["o"], non_blocking=True)
+                down_ev[i].record(down)
+        stream.wait_event(down_ev[n - 1])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1)
 
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    e2e_run(3)
     barrier(world)
-    for i in range(steps):
-        e_ev[i][0].record(stream)
-        e2e_step()
-        e_ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev), world)
+    e2e_ms = max_over_ranks(e2e_run(steps), world)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv)) + (hoffs.numel() * 4 if hoffs is not None else 0)
-    d2h = hout.numel() * hout.element_size()
+    d2h = houts[0].numel() * houts[0].element_size()
     e2e = {"value": all_flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h}
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / steps,
+           "pipeline": "each step uploads its inputs and downloads its output (pinned host memory); "
+                       "double-buffered on two copy streams, so step i+1's upload and step i-1's download "
+                       "overlap step i's kernels"}
+    del bufs, houts
     if la.llama_attn_get_device_error() != 0:
         raise RuntimeError("device error word set during the benchmark")
     cpu = None
