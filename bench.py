@@ -742,17 +742,44 @@ def run_decode(args, la, dev, world, rank, hbm_peak, peak_kind):
     }
 
 
+def code_sha1(text: str) -> str:
+    """sha1 of C/C++/CUDA source with its comments, trailing blanks and empty
+    lines removed, so that editing a comment leaves it unchanged while any change
+    to the code (including whitespace inside a line) changes it."""
+    import hashlib
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":  # string or character literal, copied with its escapes
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = [ln.rstrip() for ln in "".join(out).split("\n")]
+    return hashlib.sha1("\n".join(ln for ln in lines if ln).encode()).hexdigest()
+
+
 def load_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu record, or None when there is
-    no record for this kernel and workload or the kernel source has changed
-    since the counters were taken."""
-    import hashlib
+    no record for this kernel and workload or the kernel's code (comments aside)
+    has changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)[kernel][workload]
-        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
-            if hashlib.sha1(f.read()).hexdigest() != rec["source_sha1"]:
+        with open(os.path.join(ROOT, rec["source"])) as f:
+            if code_sha1(f.read()) != rec["code_sha1"]:
                 return None
         return rec["bytes"]
     except Exception:

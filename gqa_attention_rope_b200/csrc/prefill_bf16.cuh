@@ -8,7 +8,8 @@
 //               2-stage K ring and V tiles through a 1-stage V ring, issued in
 //               the order K0, K1, V0, K2, V1, ..., so each K tile is loaded
 //               one tile ahead of its S MMAs and each V tile while the softmax
-//               of its tile runs.
+//               of its tile runs. It also claims the items and publishes each
+//               one's fields in a shared-memory ring.
 //   warp 1      TMEM owner; one thread issues S_h = Q_h K_j^T (M=128, N=128,
 //               K=128; fp32 accumulators in TMEM)
 //   warp 2      one thread issues O_h += P_h V_j (P from shared memory, V MN-major).
@@ -17,8 +18,7 @@
 //               has completed) would otherwise leave the tensor pipe idle; with
 //               S and PV issued from different threads one thread's waits
 //               overlap the other's MMAs.
-//   Registers: the four role warps (one warpgroup) hold 64 each and give the
-//   rest to the eight softmax warps, which hold 216 each (setmaxnreg).
+//   warp 3      one thread stores each finished output tile with TMA.
 //   warps 4-7   softmax for head slot 0, warps 8-11 for slot 1: thread = query
 //               row = TMEM lane. Rotates its Q row in shared memory (RoPE at the
 //               row's document position), then per KV tile: S from TMEM ->
@@ -26,11 +26,18 @@
 //               shared memory, running sum; O in TMEM is rescaled only when the
 //               running max grows by more than 2^8 (exact: the final 1/l uses the
 //               same reference max); epilogue O/l -> bf16 -> TMA store.
+//   Registers: the four role warps (one warpgroup) hold 64 each and give the
+//   rest to the eight softmax warps, which hold 216 each (setmaxnreg).
 //
 // TMEM columns: S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
 // Shared memory (1024-aligned): Q_0, Q_1 (32 KB each), K ring 2 x 32 KB, V ring
-// 32 KB, P_0, P_1 (32 KB each), barriers. Every 32 KB tile is two 64-column halves of
-// 128 rows x 128 B in the 128B-swizzled layout TMA writes.
+// 32 KB, P_0, P_1 (32 KB each), barriers and the item ring. Every 32 KB tile is
+// two 64-column halves of 128 rows x 128 B in the 128B-swizzled layout TMA
+// writes.
+//
+// Items run heaviest first (the last query tiles first); when the keys and
+// values are far larger than L2 they run KV group by KV group instead, heaviest
+// first inside each group (see item_of).
 //
 // KV tiles run from the tile holding the document start of the first query
 // row to the diagonal tile; tiles entirely before that start are never loaded
@@ -121,8 +128,9 @@ __device__ __forceinline__ uint64_t kdesc(uint32_t saddr) { return umma_desc_sw1
 __device__ __forceinline__ uint64_t vdesc(uint32_t saddr) { return umma_desc_sw128(saddr, HALF, 1024); }
 
 // One work item: a 128-row query tile of batch row b for query heads
-// h0 .. h0 + NH - 1 (all of KV group g). Items are numbered heaviest first
-// (highest query tile first); every role of a CTA derives the same items.
+// h0 .. h0 + NH - 1 (all of KV group g). item_of numbers them heaviest first
+// (highest query tile first), over all groups or inside each KV group in turn;
+// the producer computes each item's fields once and publishes them.
 struct Item {
   int b, h0, g, q0, ds_last, kv_t0, n_kv;
   int64_t rowbase;
@@ -168,8 +176,9 @@ __device__ __forceinline__ Item item_of(int item, const Params& p) {
 }
 
 // Persistent: one CTA per SM. Its first item is blockIdx.x; later ones are
-// claimed with an atomic counter (gridDim.x + counter), so items, numbered
-// heaviest first, are handed out first-come (longest-processing-time-first).
+// claimed with an atomic counter (gridDim.x + counter), so items are handed
+// out first-come in item_of's order (longest-processing-time-first, inside each
+// KV group when the items run group by group).
 // The producer publishes each claimed item id in an 8-entry shared-memory ring
 // as soon as it is claimed (well before its Q tiles are loaded); -1 ends every
 // role's loop.
