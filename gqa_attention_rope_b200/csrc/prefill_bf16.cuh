@@ -339,12 +339,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int s = 0; s < p.NH; ++s)
             for (int hf = 0; hf < 2; ++hf)
               tma_load_4d(sbase + OFF_Q + s * TILE + hf * HALF, &tm_q, bar(B_Q_FULL), hf * 64, I.h0 + s, I.q0, I.b);
+          // The item's first K tiles go out before the next item is claimed and
+          // published (an atomic and two document-start reads): the first S
+          // MMAs wait for them, the consumers of the next item's fields not yet.
+          ok = load_k(I.g, I.kv_t0 * BN, I.b);
+          if (ok && I.n_kv > 1) ok = load_k(I.g, (I.kv_t0 + 1) * BN, I.b);
           item = next_item;
           next_item = (item < n_items) ? atomicAdd(p.sched, 1) + static_cast<int>(gridDim.x) : n_items;
           publish(it + 1, item < n_items ? item : -1);
           prefetch_rows(item);
-          ok = load_k(I.g, I.kv_t0 * BN, I.b);
-          for (int j = 1; ok && j < I.n_kv; ++j)
+          if (ok && I.n_kv > 1) ok = load_v(I.g, I.kv_t0 * BN, I.b);
+          for (int j = 2; ok && j < I.n_kv; ++j)
             ok = load_k(I.g, (I.kv_t0 + j) * BN, I.b) && load_v(I.g, (I.kv_t0 + j - 1) * BN, I.b);
           if (ok) ok = load_v(I.g, (I.kv_t0 + I.n_kv - 1) * BN, I.b);
           if (!ok) {
@@ -534,30 +539,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const float4 st0 = __ldg(step), st1 = __ldg(step + 1);
           float4 c0 = make_float4(1.f, 0.f, 1.f, 0.f), c1 = c0;
           int pos_prev = -4;
-  #pragma unroll 4
-          for (int i = 0; i < 16; ++i) {
-            const int src = 2 * i + (lane >> 4);  // lane of the warp that owns the row
-            const int rr = wq * 32 + src;
-            const int pos = __shfl_sync(0xffffffffu, qi_c - ds_i, src);
-            if (pos == pos_prev + 2) {
-              c0 = make_float4(c0.x * st0.x - c0.y * st0.y, c0.y * st0.x + c0.x * st0.y,
-                               c0.z * st0.z - c0.w * st0.w, c0.w * st0.z + c0.z * st0.w);
-              c1 = make_float4(c1.x * st1.x - c1.y * st1.y, c1.y * st1.x + c1.x * st1.y,
-                               c1.z * st1.z - c1.w * st1.w, c1.w * st1.z + c1.z * st1.w);
-            } else {
-              const float4* tab = p.rope_tab + static_cast<int64_t>(pos) * 32 + 2 * ch;
-              c0 = __ldg(tab);
-              c1 = __ldg(tab + 1);
+          const int pos_own = qi_c - ds_i;
+          const uint32_t hoff = (ch >> 3) * HALF;
+          // Four of the half-warp's rows at a time: their chunks are all read
+          // before any is written back, so one shared-memory round trip (slow
+          // here: the last PV MMAs and the next item's TMA loads share the
+          // bandwidth) serves four rows.
+  #pragma unroll 1
+          for (int i0 = 0; i0 < 16; i0 += 4) {
+            uint4 x[4];
+  #pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int rr = wq * 32 + 2 * (i0 + u) + (lane >> 4);
+              x[u] = *reinterpret_cast<const uint4*>(qtile + hoff + sw128_off(rr, ch & 7));
             }
-            pos_prev = pos;
-            if (I.q0 + rr < p.S) {
-              uint4* ptr = reinterpret_cast<uint4*>(qtile + (ch >> 3) * HALF + sw128_off(rr, ch & 7));
-              uint4 x = *ptr;
-              x.x = rope_rotate_pair(x.x, c0.x, c0.y);
-              x.y = rope_rotate_pair(x.y, c0.z, c0.w);
-              x.z = rope_rotate_pair(x.z, c1.x, c1.y);
-              x.w = rope_rotate_pair(x.w, c1.z, c1.w);
-              *ptr = x;
+  #pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int src = 2 * (i0 + u) + (lane >> 4);  // lane of the warp that owns the row
+              const int pos = __shfl_sync(0xffffffffu, pos_own, src);
+              if (pos == pos_prev + 2) {
+                c0 = make_float4(c0.x * st0.x - c0.y * st0.y, c0.y * st0.x + c0.x * st0.y,
+                                 c0.z * st0.z - c0.w * st0.w, c0.w * st0.z + c0.z * st0.w);
+                c1 = make_float4(c1.x * st1.x - c1.y * st1.y, c1.y * st1.x + c1.x * st1.y,
+                                 c1.z * st1.z - c1.w * st1.w, c1.w * st1.z + c1.z * st1.w);
+              } else {
+                const float4* tab = p.rope_tab + static_cast<int64_t>(pos) * 32 + 2 * ch;
+                c0 = __ldg(tab);
+                c1 = __ldg(tab + 1);
+              }
+              pos_prev = pos;
+              x[u].x = rope_rotate_pair(x[u].x, c0.x, c0.y);
+              x[u].y = rope_rotate_pair(x[u].y, c0.z, c0.w);
+              x[u].z = rope_rotate_pair(x[u].z, c1.x, c1.y);
+              x[u].w = rope_rotate_pair(x[u].w, c1.z, c1.w);
+            }
+  #pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int rr = wq * 32 + 2 * (i0 + u) + (lane >> 4);
+              if (I.q0 + rr < p.S) *reinterpret_cast<uint4*>(qtile + hoff + sw128_off(rr, ch & 7)) = x[u];
             }
           }
         }
