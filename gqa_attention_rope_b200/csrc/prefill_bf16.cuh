@@ -645,10 +645,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int c = 0; c < 128; c += 2) {
             float x0, x1;
             f2_unpack(f2_fma(f2_pack(sv[c], sv[c + 1]), sl2x2, negmx2), x0, x1);
-            // one pair in eight goes through the FMA-pipe polynomial, the rest
-            // through MUFU (with the register split, 1/8 and 1/4 measured best;
-            // larger shares cost more FMA and ALU issue than the MUFU time saved)
-            const bool poly = (c & 14) == 14;
+            // one pair in sixteen goes through the FMA-pipe polynomial, the rest
+            // through MUFU (1/16 measured best on all three prefill workloads,
+            // 1/8 within 1.5%; 1/4 and larger shares cost more FMA and ALU
+            // issue than the MUFU time saved)
+            const bool poly = (c & 30) == 30;
             const float p0 = poly ? ex2_poly(x0) : ex2_approx(x0);
             const float p1 = poly ? ex2_poly(x1) : ex2_approx(x1);
             if (c & 2) rsb = f2_add(rsb, f2_pack(p0, p1));
